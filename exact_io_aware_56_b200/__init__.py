@@ -1,0 +1,11 @@
+"""Exact IO-aware attention (forward and backward) for B200 / sm_100a.
+
+The compute runs in ``libfa.so`` (hand-written CUDA for sm_100a behind a C
+ABI, declared in ``include/fa.h``). :mod:`exact_io_aware_56_b200.fa` is the
+thin ctypes binding with the same entry-point names; it raises if the library
+is missing or no CUDA device is present, and there is no CPU fallback.
+"""
+
+from .inputs import WORKLOADS, Workload, make_inputs, sample_rows, to_f64  # noqa: F401
+
+__all__ = ["WORKLOADS", "Workload", "make_inputs", "sample_rows", "to_f64"]

@@ -1,0 +1,254 @@
+"""Exact attention in float64 on the CPU: the definition, written out.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring). Nothing on the product
+path may import this module.
+
+Shapes follow the kernels' layout: ``q`` is ``[B, Hq, N, d]``, ``k`` and ``v``
+are ``[B, Hkv, N, d]``, ``dout`` is like ``q``. All arrays are float64.
+
+What is computed (FlashAttention: IO-aware exact attention, "NAIVE" box of the
+"NAIVE ATTENTION vs FLASHATTENTION" diagram): S = scale * Q K^T, P =
+softmax(S) row by row, O = P V. The "FLASH" box of the same diagram, and the
+"Four ideas" list (item "Online softmax"), state that the tiled online form
+reaches the same O exactly, and that one logsumexp per query row is kept for
+the backward pass; that value is L_i = log sum_j exp(S_ij) (natural log).
+
+Readings taken where the pages are silent (each is listed in the design
+notes):
+
+* The softmax scale multiplies Q K^T before the mask and the softmax.
+* Causal masking hides key j from query i when j > i (queries and keys have
+  the same length, so top-left and bottom-right alignment agree).
+* Grouped-query attention (the "PREFILL PATH" diagram's notes on decode and
+  the explainer's "Use with GQA") groups query heads contiguously: query head
+  h reads KV head h // (Hq // Hkv).
+* The FLASH box prints the loop body but not the last step; the plain reading
+  is O <- O / l and L = m + ln l.
+* The backward pass (the "Four ideas" item "Recomputation in the backward
+  pass") is the textbook gradient of the definition: dV = P^T dO,
+  dP = dO V^T, D_i = sum_j P_ij dP_ij, dS = P o (dP - D), dQ = scale dS K,
+  dK = scale dS^T Q, summed over the query heads that share a KV head.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# Rows of S materialised at once by the blocked helpers. Only bounds memory;
+# each row's arithmetic is unchanged by it.
+_ROW_CHUNK = 512
+
+
+def kv_head_of(hq: int, Hq: int, Hkv: int) -> int:
+    """KV head read by query head ``hq``: contiguous groups of Hq/Hkv heads."""
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return hq // (Hq // Hkv)
+
+
+def _check(q, k, v):
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, Hq, N, d = q.shape
+    if k.shape[0] != B or k.shape[2] != N or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, d] with q's B, N, d")
+    if Hq % k.shape[1] != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return B, Hq, k.shape[1], N, d
+
+
+def _scores(qrows, kmat, scale, causal, row_ids):
+    """Rows of S = scale * Q K^T, with masked entries set to -inf.
+
+    ``row_ids`` are the query positions of ``qrows`` (used by the causal mask).
+    """
+    S = scale * (qrows @ kmat.T)
+    if causal:
+        cols = np.arange(kmat.shape[0])
+        S[cols[None, :] > np.asarray(row_ids)[:, None]] = -np.inf
+    return S
+
+
+def _softmax_rows(S):
+    """Two-pass softmax of each row (max, then normalised exponentials).
+
+    Returns P and the row logsumexp L = m + ln(sum exp(S - m)).
+    """
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    l = E.sum(axis=1, keepdims=True)
+    return E / l, (m + np.log(l))[:, 0]
+
+
+def attn_fwd_ref(q, k, v, causal: bool, scale: float):
+    """Naive forward: S and P materialised, two-pass softmax, O = P V.
+
+    FlashAttention: IO-aware exact attention, "NAIVE" box of the "NAIVE
+    ATTENTION vs FLASHATTENTION" diagram (S = Q K^T, P = softmax(S),
+    O = P V), plus the logsumexp of the "FLASH" box.
+
+    Returns ``(O, L)`` with O like ``q`` and L ``[B, Hq, N]``.
+    """
+    B, Hq, Hkv, N, d = _check(q, k, v)
+    O = np.empty_like(q, dtype=np.float64)
+    L = np.empty((B, Hq, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            for r0 in range(0, N, _ROW_CHUNK):
+                rows = np.arange(r0, min(N, r0 + _ROW_CHUNK))
+                S = _scores(q[b, h, rows], k[b, g], scale, causal, rows)
+                P, Lr = _softmax_rows(S)
+                O[b, h, rows] = P @ v[b, g]
+                L[b, h, rows] = Lr
+    return O, L
+
+
+def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
+                        block_q: int = 128, block_k: int = 128):
+    """Tiled forward with the online softmax, in the pages' order.
+
+    FlashAttention: IO-aware exact attention, "FLASH" box of the "NAIVE
+    ATTENTION vs FLASHATTENTION" diagram: for each Q block start from
+    O = 0, m = -inf, l = 0; for each K, V block form the score tile, raise
+    the running max, rescale l and O by e^(m - m_new), add the new block's
+    exponentials, and move m forward. After the last block O is divided by
+    l and L = m + ln l is kept (the box's final line; the divide is the
+    plain reading of "write O once"). Only m, l and O persist between
+    blocks ("PREFILL PATH" diagram: "Only m, l, O stay"); no N x N array is
+    built. Returns ``(O, L)`` like :func:`attn_fwd_ref`.
+    """
+    B, Hq, Hkv, N, d = _check(q, k, v)
+    if block_q < 1 or block_k < 1:
+        raise ValueError("block sizes must be positive")
+    O_out = np.empty_like(q, dtype=np.float64)
+    L_out = np.empty((B, Hq, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            for i0 in range(0, N, block_q):
+                rows = np.arange(i0, min(N, i0 + block_q))
+                Qb = q[b, h, rows]
+                O = np.zeros((len(rows), d))
+                m = np.full(len(rows), -np.inf)
+                l = np.zeros(len(rows))
+                for j0 in range(0, N, block_k):
+                    cols = np.arange(j0, min(N, j0 + block_k))
+                    S = scale * (Qb @ k[b, g, cols].T)
+                    if causal:
+                        S[cols[None, :] > rows[:, None]] = -np.inf
+                    m_new = np.maximum(m, S.max(axis=1))
+                    # A row whose blocks so far are all masked keeps m = -inf;
+                    # its factors are then defined as 1 (nothing to rescale).
+                    safe = np.where(np.isneginf(m_new), 0.0, m_new)
+                    alpha = np.where(np.isneginf(m_new), 1.0, np.exp(m - safe))
+                    E = np.exp(S - safe[:, None])
+                    l = alpha * l + E.sum(axis=1)
+                    O = alpha[:, None] * O + E @ v[b, g, cols]
+                    m = m_new
+                O_out[b, h, rows] = O / l[:, None]
+                L_out[b, h, rows] = m + np.log(l)
+    return O_out, L_out
+
+
+def attn_bwd_ref(q, k, v, dout, causal: bool, scale: float):
+    """Gradients of sum(dout * O) with respect to q, k, v.
+
+    The pages state only that the backward pass rebuilds P from Q, K and L
+    ("Four ideas", item "Recomputation in the backward pass"; blog section
+    "Recomputation in the Backward Pass"). The formulas are the textbook
+    gradient of softmax attention, materialised here row block by row block:
+    P is rebuilt from S with the row logsumexp, dV = P^T dO, dP = dO V^T,
+    D_i = sum_j P_ij dP_ij, dS = P o (dP - D), dQ = scale dS K and
+    dK = scale dS^T Q. KV heads shared by several query heads sum the
+    contributions of all of them.
+
+    Returns ``(dq, dk, dv)`` shaped like ``q``, ``k``, ``v``.
+    """
+    B, Hq, Hkv, N, d = _check(q, k, v)
+    dq = np.zeros_like(q, dtype=np.float64)
+    dk = np.zeros_like(k, dtype=np.float64)
+    dv = np.zeros_like(v, dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            for r0 in range(0, N, _ROW_CHUNK):
+                rows = np.arange(r0, min(N, r0 + _ROW_CHUNK))
+                S = _scores(q[b, h, rows], k[b, g], scale, causal, rows)
+                P, _ = _softmax_rows(S)
+                dO = dout[b, h, rows]
+                dv[b, g] += P.T @ dO
+                dP = dO @ v[b, g].T
+                D = (P * dP).sum(axis=1, keepdims=True)
+                dS = P * (dP - D)
+                dq[b, h, rows] = scale * (dS @ k[b, g])
+                dk[b, g] += scale * (dS.T @ q[b, h, rows])
+    return dq, dk, dv
+
+
+def attn_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
+    """O and L of query head ``h`` of batch ``b`` at the given query rows only.
+
+    Same arithmetic as :func:`attn_fwd_ref` restricted to some rows (each row
+    of the definition depends only on its own row of S). Returns
+    ``(O_rows [len(rows), d], L_rows [len(rows)])``.
+    """
+    _, Hq, Hkv, _, _ = _check(q, k, v)
+    g = kv_head_of(h, Hq, Hkv)
+    rows = np.asarray(rows)
+    O = np.empty((len(rows), q.shape[3]))
+    L = np.empty(len(rows))
+    for c0 in range(0, len(rows), _ROW_CHUNK):
+        rr = rows[c0:c0 + _ROW_CHUNK]
+        S = _scores(q[b, h, rr], k[b, g], scale, causal, rr)
+        P, Lr = _softmax_rows(S)
+        O[c0:c0 + len(rr)] = P @ v[b, g]
+        L[c0:c0 + len(rr)] = Lr
+    return O, L
+
+
+def attn_bwd_rows(q, k, v, dout, causal: bool, scale: float, b: int, h: int, rows):
+    """dQ of query head ``h`` of batch ``b`` at the given query rows only.
+
+    dQ_i = scale * sum_j P_ij (dP_ij - D_i) K_j needs only row i of P and dP
+    (D_i is a sum along that same row), so it is exact for a subset of rows.
+    """
+    _, Hq, Hkv, _, _ = _check(q, k, v)
+    g = kv_head_of(h, Hq, Hkv)
+    rows = np.asarray(rows)
+    dq = np.empty((len(rows), q.shape[3]))
+    for c0 in range(0, len(rows), _ROW_CHUNK):
+        rr = rows[c0:c0 + _ROW_CHUNK]
+        S = _scores(q[b, h, rr], k[b, g], scale, causal, rr)
+        P, _ = _softmax_rows(S)
+        dP = dout[b, h, rr] @ v[b, g].T
+        D = (P * dP).sum(axis=1, keepdims=True)
+        dq[c0:c0 + len(rr)] = scale * ((P * (dP - D)) @ k[b, g])
+    return dq
+
+
+def attn_bwd_kv_rows(q, k, v, dout, causal: bool, scale: float, b: int, g: int, keys):
+    """dK and dV of KV head ``g`` of batch ``b`` at the given key rows only.
+
+    Column j of P and dS depends on every query row's logsumexp and D_i, so
+    all query rows of every query head sharing KV head ``g`` are rebuilt
+    (row block by row block) and only the requested key columns are kept.
+    Returns ``(dk_rows [len(keys), d], dv_rows [len(keys), d])``.
+    """
+    _, Hq, Hkv, N, d = _check(q, k, v)
+    keys = np.asarray(keys)
+    r = Hq // Hkv
+    dk = np.zeros((len(keys), d))
+    dv = np.zeros((len(keys), d))
+    for h in range(g * r, (g + 1) * r):
+        for r0 in range(0, N, _ROW_CHUNK):
+            rows = np.arange(r0, min(N, r0 + _ROW_CHUNK))
+            S = _scores(q[b, h, rows], k[b, g], scale, causal, rows)
+            P, _ = _softmax_rows(S)
+            dO = dout[b, h, rows]
+            dP = dO @ v[b, g].T
+            D = (P * dP).sum(axis=1, keepdims=True)
+            dS = P * (dP - D)
+            dv += P[:, keys].T @ dO
+            dk += scale * (dS[:, keys].T @ q[b, h, rows])
+    return dk, dv

@@ -1,0 +1,108 @@
+"""Planted mistakes in the oracle must be caught by its pins.
+
+Each mutation patches the oracle on the CPU (never the CUDA path) with a
+plausible error: an off-by-one causal mask, a dropped scale, a missing
+normalisation, the wrong logarithm base, a flipped sign, swapped or
+mis-summed gradients. The test passes only if at least one pin in
+``test_oracle_pins`` fails under the mutation.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention as A
+
+from . import test_oracle_pins as pins
+
+FWD_CHECKS = [pins.check_brute_force, pins.check_online_equals_two_pass, pins.check_rows_sum_to_one,
+              pins.check_constant_v, pins.check_zero_q, pins.check_causal_row0,
+              pins.check_permutation_invariance]
+
+
+def _fails(checks, **kw):
+    for c in checks:
+        try:
+            c(**kw)
+        except AssertionError:
+            return True
+    return False
+
+
+_orig_scores = A._scores
+_orig_softmax = A._softmax_rows
+
+
+def scores_mask_off_by_one(qrows, kmat, scale, causal, row_ids):
+    S = scale * (qrows @ kmat.T)
+    if causal:
+        cols = np.arange(kmat.shape[0])
+        S[cols[None, :] >= np.asarray(row_ids)[:, None] + 2] = -np.inf
+    return S
+
+
+def scores_no_scale(qrows, kmat, scale, causal, row_ids):
+    return _orig_scores(qrows, kmat, 1.0, causal, row_ids)
+
+
+def scores_transposed(qrows, kmat, scale, causal, row_ids):
+    # Uses K's rows in reverse order (a wrong index into K).
+    return _orig_scores(qrows, kmat[::-1], scale, causal, row_ids)
+
+
+def softmax_unnormalised(S):
+    m = S.max(axis=1, keepdims=True)
+    E = np.exp(S - m)
+    return E, (m + np.log(E.sum(axis=1, keepdims=True)))[:, 0]
+
+
+def softmax_log2(S):
+    P, L = _orig_softmax(S)
+    return P, L / np.log(2.0)
+
+
+@pytest.mark.parametrize("name,target,repl", [
+    ("causal mask off by one", "_scores", scores_mask_off_by_one),
+    ("scale dropped", "_scores", scores_no_scale),
+    ("key rows misindexed", "_scores", scores_transposed),
+    ("softmax not normalised", "_softmax_rows", softmax_unnormalised),
+    ("logsumexp in base 2", "_softmax_rows", softmax_log2),
+])
+def test_forward_mutation_is_caught(monkeypatch, name, target, repl):
+    monkeypatch.setattr(A, target, repl)
+    assert _fails(FWD_CHECKS), name
+
+
+def _wrap_bwd(kind):
+    ref = oracle.attn_bwd_ref
+
+    def bwd(q, k, v, dout, causal, scale):
+        dq, dk, dv = ref(q, k, v, dout, causal, scale)
+        if kind == "dq sign":
+            return -dq, dk, dv
+        if kind == "dk no scale":
+            return dq, dk / scale, dv
+        if kind == "dk dv swapped":
+            return dq, dv, dk
+        if kind == "gqa not summed":
+            # Keeps only the first query head's share of each KV head.
+            r = q.shape[1] // k.shape[1]
+            if r == 1:
+                return dq, dk, dv
+            q1 = q.copy(); dout1 = dout.copy()
+            for h in range(q.shape[1]):
+                if h % r:
+                    dout1[:, h] = 0.0
+            _, dk1, dv1 = ref(q1, k, v, dout1, causal, scale)
+            return dq, dk1, dv1
+        raise KeyError(kind)
+    return bwd
+
+
+@pytest.mark.parametrize("kind", ["dq sign", "dk no scale", "dk dv swapped", "gqa not summed"])
+def test_backward_mutation_is_caught(kind):
+    assert _fails([pins.check_backward_fd], bwd=_wrap_bwd(kind)), kind
+
+
+def test_unmutated_oracle_passes_all_checks():
+    assert not _fails(FWD_CHECKS + [pins.check_backward_fd])
