@@ -1,0 +1,207 @@
+// C-ABI layer of libfa: argument checks, device check, TMA tensor maps,
+// watchdog word, status strings. Declared in include/fa.h.
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Device error word written by the kernels' watchdog.
+__device__ unsigned int g_err_word;
+
+std::atomic<uint64_t> g_budget_ns{2000000000ull};
+std::atomic<int> g_fault{0};
+thread_local char t_cuda_msg[256] = "no CUDA error recorded";
+
+struct DevState {
+  std::once_flag once;
+  bool supported = false;
+  unsigned int* err = nullptr;
+};
+DevState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+int record_cuda(cudaError_t e) {
+  snprintf(t_cuda_msg, sizeof(t_cuda_msg), "CUDA error %d: %s", static_cast<int>(e), cudaGetErrorString(e));
+  return FA_ERR_CUDA;
+}
+
+// Checks the current device once: compute capability 10.0 (sm_100a) and the
+// address of its error word. Returns FA_OK or an error status.
+int device_state(DevState** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  DevState& st = g_dev[dev];
+  std::call_once(st.once, [&] {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return;
+    if (major != 10 || minor != 0) return;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return;
+    st.err = static_cast<unsigned int*>(p);
+    st.supported = true;
+  });
+  if (!st.supported) return FA_ERR_UNSUPPORTED;
+  *out = &st;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int Hq, int Hkv, int N, int d, int causal, float scale) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0) return FA_ERR_INVALID_ARGUMENT;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  // Index arithmetic limits: (B*Hq) fits the grid and a TMA coordinate; the
+  // element count of one tensor stays below 2^40.
+  const long long bh = static_cast<long long>(B) * Hq;
+  if (bh > (1LL << 30)) return FA_ERR_UNSUPPORTED;
+  if (bh * N * d >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+LaunchCtl make_ctl(const DevState* st) {
+  LaunchCtl c;
+  c.err = st->err;
+  c.budget_ns = g_budget_ns.load(std::memory_order_relaxed);
+  c.fault = g_fault.load(std::memory_order_relaxed);
+  return c;
+}
+
+}  // namespace
+
+bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(cols) * 2 * rows};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+           int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARGUMENT;
+  int rc = check_shape(B, Hq, Hkv, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  DevState* st = nullptr;
+  if ((rc = device_state(&st)) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (!encode_tile_map(&tq, q, d, N, B * Hq, 128) || !encode_tile_map(&tk, k, d, N, B * Hkv, 128) ||
+      !encode_tile_map(&tv, v, d, N, B * Hkv, 128))
+    return FA_ERR_UNSUPPORTED;
+  AttnShape s{B, Hq, Hkv, N, d, causal, scale};
+  cudaError_t e = launch_fwd(s, tq, tk, tv, o, lse, make_ctl(st), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  if (check_shape(B, Hq, Hkv, N, d, 0, 1.f) != FA_OK) return 0;
+  AttnShape s{B, Hq, Hkv, N, d, 0, 1.f};
+  return bwd_workspace_bytes(s);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARGUMENT;
+  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_INVALID_ARGUMENT;
+  int rc = check_shape(B, Hq, Hkv, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  AttnShape s{B, Hq, Hkv, N, d, causal, scale};
+  if (workspace_bytes < bwd_workspace_bytes(s)) return FA_ERR_INVALID_ARGUMENT;
+  DevState* st = nullptr;
+  if ((rc = device_state(&st)) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_tile_map(&tq, q, d, N, B * Hq, 128) || !encode_tile_map(&tk, k, d, N, B * Hkv, 128) ||
+      !encode_tile_map(&tv, v, d, N, B * Hkv, 128) || !encode_tile_map(&tdo, dout, d, N, B * Hq, 128))
+    return FA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_bwd(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, make_ctl(st),
+                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK:
+      return "ok";
+    case FA_ERR_INVALID_ARGUMENT:
+      return "invalid argument (null or misaligned pointer, non-positive size, bad causal flag, "
+             "non-finite or non-positive scale, or workspace too small)";
+    case FA_ERR_UNSUPPORTED:
+      return "unsupported (head dim not 64/128, Hq not a multiple of Hkv, size limit, or device is not "
+             "compute capability 10.0)";
+    case FA_ERR_CUDA:
+      return t_cuda_msg;
+    case FA_ERR_TIMEOUT:
+      return "a kernel wait ran past the watchdog budget and the kernel gave up";
+    default:
+      return "unknown status";
+  }
+}
+
+int fa_check_device_error(void* stream) {
+  DevState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != FA_OK) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return record_cuda(e);
+  unsigned int word = 0;
+  e = cudaMemcpy(&word, st->err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return record_cuda(e);
+  if (word == 0) return FA_OK;
+  e = cudaMemset(st->err, 0, sizeof(word));
+  if (e != cudaSuccess) return record_cuda(e);
+  e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return record_cuda(e);
+  return FA_ERR_TIMEOUT;
+}
+
+void fa_set_watchdog_ns(uint64_t ns) { g_budget_ns.store(ns < 1000000ull ? 1000000ull : ns); }
+
+// Test hook, declared in include/fa_test.h: selects a deliberate stall
+// (1 = the forward producer never loads the first K tile) so that the
+// watchdog path can be exercised without faulting the GPU.
+void fa_test_set_fault(int code) { g_fault.store(code); }
+
+}  // extern "C"

@@ -1,0 +1,390 @@
+// Forward attention kernel for sm_100a.
+//
+// Computes O = softmax(scale * Q K^T [+ causal mask]) V and the row
+// logsumexp L, tile by tile, without writing the N x N scores anywhere
+// (FlashAttention: IO-aware exact attention, "FLASH" box of the "NAIVE
+// ATTENTION vs FLASHATTENTION" diagram, and the "PREFILL PATH" diagram:
+// a 128-row Q block stays on chip, 128-column K/V blocks stream through
+// shared memory and are dropped, only m, l and O persist, O is written once
+// together with one logsumexp per row).
+//
+// One CTA owns two 128-row Q tiles of one (batch, query head) and streams
+// the K/V tiles of its KV head once for both. Warp roles:
+//   warps 0-3   softmax for Q tile 0, warps 4-7 for Q tile 1: one thread
+//               per query row (warp w reads tensor-memory lanes 32*(w%4)..).
+//   warp 8      TMA producer: Q tiles once, then K_j / V_j into a ring of
+//               shared-memory stages (mbarrier full / empty pairs).
+//   warp 9      tensor-memory owner and MMA issuer (one thread):
+//               S_t = Q_t K_j^T (tcgen05, both operands in shared memory),
+//               O_t += P_t V_j (tcgen05, P_t read from tensor memory).
+//   warps 10-11 idle (keep the third warpgroup whole).
+// The softmax is the online form of the "Four ideas" list (item "Online
+// softmax"): running max m, running sum l, O rescaled by e^(m - m_new)
+// when the max grows.
+//
+// Tensor memory (512 columns x 128 lanes, fp32):
+//   [0,128) S_0 | [128,256) S_1 | [256,256+D) O_0 | [256+D,256+2D) O_1
+// P_t (bf16, two per column) overwrites the first 64 columns of S_t.
+//
+// Ordering argument used by the softmax warps: the MMA thread issues, for
+// each tile t, S_t^(j+1) after O_t += P_t^j V_j, and tcgen05 operations
+// complete in issue order, so once S_t^(j+1) is signalled complete the O_t
+// accumulator holds every earlier product and may be rescaled in place
+// until P_t^(j+1) is handed back.
+//
+// The exponentials are base 2: scores are scaled by scale*log2(e), and
+// L = (m + log2 l) * ln 2. The rescale of O is lazy: a warp rescales only
+// when some row's max grew by more than 8 (a factor 256), otherwise every
+// row keeps its stale max, which changes no result because l and O share it.
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;   // query rows per Q tile
+constexpr int kBN = 128;   // keys per K/V tile
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kBoxBytes = kBN * 64 * 2;       // one 64-column TMA box of a 128-row tile
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kTileBytes = kBoxBytes * kBoxes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kSmemBytes > 114 * 1024, "one CTA per SM (owns all tensor memory)");
+};
+
+struct FwdArgs {
+  __nv_bfloat16* o;
+  float* lse;
+  int N, Hq, Hkv, BH, n_pairs, nk;
+  float scale_log2;
+  LaunchCtl ctl;
+};
+
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t s_full[2], p_ready[2], o_final[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using C = FwdCfg<D>;
+  constexpr int ST = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::kOffBar);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: (batch*head, pair of Q tiles). The heaviest pairs (largest
+  // query index, most K/V tiles when causal) get the lowest block indices so
+  // they start first; heads sharing a KV head are adjacent.
+  const int bh = blockIdx.x % a.BH;
+  const int pair = a.n_pairs - 1 - blockIdx.x / a.BH;
+  const int h = bh % a.Hq;
+  const int b = bh / a.Hq;
+  const int kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
+  const int q0 = pair * 2 * kBM;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) n_t[t] = CAUSAL ? min(a.nk, 2 * pair + t + 1) : a.nk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_ready[t], kBM);
+      mbar_init(&bars->o_final[t], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const Watch w{&bars->abort, a.ctl.err, a.ctl.budget_ns};
+
+  const uint32_t sQ = smem_u32(smem + C::kOffQ);
+  const uint32_t sK = smem_u32(smem + C::kOffK);
+  const uint32_t sV = smem_u32(smem + C::kOffV);
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int k_last[ST], v_last[ST];
+#pragma unroll
+      for (int s = 0; s < ST; ++s) k_last[s] = v_last[s] = -1;
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::kTileBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_3d(&tmQ, &bars->q_full, smem + C::kOffQ + t * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                      q0 + t * kBM, bh);
+      const int n = n_t[1];
+      for (int j = 0; j < n; ++j) {
+        const int s = j % ST;
+        const int u = j / ST;
+        if (j >= ST && !wait_bar(&bars->kv_empty[s], (u - 1) & 1, w)) break;
+        if (!(a.ctl.fault == 1 && j == 0)) {
+          mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+#pragma unroll
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                        j * kBN, kvh);
+          k_last[s] = u;
+        }
+        mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+#pragma unroll
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                      j * kBN, kvh);
+        v_last[s] = u;
+      }
+      // Every copy issued must land before the CTA may exit.
+      drain_bar(&bars->q_full, 0, w);
+#pragma unroll
+      for (int s = 0; s < ST; ++s) {
+        if (k_last[s] >= 0) drain_bar(&bars->k_full[s], k_last[s] & 1, w);
+        if (v_last[s] >= 0) drain_bar(&bars->v_full[s], v_last[s] & 1, w);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, false, true);
+      const uint32_t tS[2] = {tmem, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qa = sQ + t * C::kTileBytes;
+        const uint32_t ka = sK + (j % ST) * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * C::kBoxBytes + (k % 4) * 32;
+          mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
+        }
+        mma_commit(&bars->s_full[t]);
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t va = sV + (j % ST) * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k)
+          mma_ts(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * 2048, C::kBoxBytes, 1024), idesc_pv,
+                 (j > 0 || k > 0) ? 1u : 0u);
+      };
+      const int n0 = n_t[0], n1 = n_t[1];
+      bool ok = wait_bar(&bars->q_full, 0, w) && wait_bar(&bars->k_full[0], 0, w);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int j = 0; ok && j < n1; ++j) {
+        const int s = j % ST;
+        const uint32_t par = (j / ST) & 1;
+        const int jn = j + 1;
+        if (j < n0) {
+          if (!(ok = wait_bar(&bars->p_ready[0], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
+          tc_fence_after();
+          issue_pv(0, j);
+          if (j == n0 - 1) mma_commit(&bars->o_final[0]);
+          if (jn < n0) {
+            if (!(ok = wait_bar(&bars->k_full[jn % ST], (jn / ST) & 1, w))) break;
+            issue_s(0, jn);
+          }
+        }
+        if (!(ok = wait_bar(&bars->p_ready[1], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(&bars->kv_empty[s]);
+        if (j == n1 - 1) mma_commit(&bars->o_final[1]);
+        if (jn < n1) {
+          if (!(ok = wait_bar(&bars->k_full[jn % ST], (jn / ST) & 1, w))) break;
+          issue_s(1, jn);
+        }
+      }
+      // All MMAs issued by this thread must finish before tensor memory is freed.
+      mma_commit(&bars->drain);
+      drain_bar(&bars->drain, 0, w);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------- softmax
+    const int t = warp >> 2;                   // Q tile of this warpgroup
+    const int quad = warp & 3;                 // tensor-memory lane quadrant
+    const int r = quad * 32 + lane;            // row within the tile
+    const int row = q0 + t * kBM + r;          // query position
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128u;
+    const uint32_t tO = tmem + lane_off + 256u + t * D;
+    const int n = n_t[t];
+    const float sl2 = a.scale_log2;
+    const int lim = CAUSAL ? min(row, a.N - 1) : a.N - 1;  // last visible key
+    float m = -CUDART_INF_F;  // running max of scale*log2(e)*s
+    float l = 0.f;            // running sum, relative to m
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[t], j & 1, w));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kBN];
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tS + c * 32, rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]);
+      }
+      if (j == n - 1) {
+        const int k0 = j * kBN;
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (k0 + i > lim) s[i] = -CUDART_INF_F;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, s[i]);
+      const float m_cand = mx * sl2;
+      if (j == 0) {
+        m = m_cand;
+      } else if (__any_sync(0xffffffffu, m_cand > m + kRescaleThreshold)) {
+        const float m_new = fmaxf(m, m_cand);
+        const float alpha = ex2(m - m_new);
+        m = m_new;
+        l *= alpha;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t oo[16];
+          tmem_ld16(tO + c * 16, oo);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) oo[i] = __float_as_uint(__uint_as_float(oo[i]) * alpha);
+          tmem_st16(tO + c * 16, oo);
+        }
+      }
+      const float neg_m = -m;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(s[c * 32 + 2 * i], sl2, neg_m));
+          const float p1 = ex2(fmaf(s[c * 32 + 2 * i + 1], sl2, neg_m));
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c * 16, pk);
+      }
+      l += sum;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_ready[t]);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->o_final[t], 0, w));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t oo[32];
+        tmem_ld32(tO + c * 32, oo);
+        uint4 v[4];
+        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pv[i] = pack_bf16x2(__uint_as_float(oo[2 * i]) * inv_l, __uint_as_float(oo[2 * i + 1]) * inv_l);
+        if (row < a.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = v[i];
+        }
+      }
+      if (row < a.N) a.lse[static_cast<size_t>(bh) * a.N + row] = (m + lg2(l)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         void* o, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  auto kern = fwd_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.N = s.N;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.BH = s.B * s.Hq;
+  a.nk = (s.N + kBN - 1) / kBN;
+  a.n_pairs = (s.N + 2 * kBM - 1) / (2 * kBM);
+  a.scale_log2 = s.scale * 1.4426950408889634f;
+  a.ctl = ctl;
+  const long long grid = static_cast<long long>(a.n_pairs) * a.BH;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       void* o, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
+  if (s.d == 64)
+    return s.causal ? launch_fwd_t<64, true>(s, tq, tk, tv, o, lse, ctl, stream)
+                    : launch_fwd_t<64, false>(s, tq, tk, tv, o, lse, ctl, stream);
+  return s.causal ? launch_fwd_t<128, true>(s, tq, tk, tv, o, lse, ctl, stream)
+                  : launch_fwd_t<128, false>(s, tq, tk, tv, o, lse, ctl, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,37 @@
+// Internal interface between the C-ABI layer (fa_api.cpp) and the kernel
+// launchers (fa_fwd.cu, fa_bwd.cu). Not installed, not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+struct AttnShape {
+  int B, Hq, Hkv, N, d;
+  int causal;
+  float scale;
+};
+
+struct LaunchCtl {
+  unsigned int* err;        // device error word (watchdog)
+  uint64_t budget_ns;       // watchdog budget per wait
+  int fault;                // test-only fault injection selector (0 = none)
+};
+
+// Encodes a 3-D bf16 tensor map over [outer][rows][cols] with a box of
+// 64 columns x box_rows rows and 128-byte swizzle. Returns false on failure.
+bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows);
+
+cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       void* o, float* lse, const LaunchCtl& ctl, cudaStream_t stream);
+
+size_t bwd_workspace_bytes(const AttnShape& s);
+
+cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const void* o, const void* dout, const float* lse, void* dq,
+                       void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,162 @@
+"""ctypes binding of libfa.so (include/fa.h): argument marshalling only.
+
+Each function takes torch CUDA tensors, checks that they have the layout the
+C ABI documents, and passes raw device pointers, sizes and the current CUDA
+stream to the library. All arithmetic happens in the CUDA kernels; there is
+no CPU fallback, and a missing library or device raises ``RuntimeError``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARGUMENT = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_TIMEOUT = 4
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libfa.so once; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_56_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.fa_fwd.restype = i
+    L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.fa_bwd_workspace_bytes.restype = sz
+    L.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_bwd.restype = i
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_check_device_error.argtypes = [vp]
+    L.fa_check_device_error.restype = i
+    L.fa_set_watchdog_ns.argtypes = [ctypes.c_uint64]
+    L.fa_set_watchdog_ns.restype = None
+    L.fa_test_set_fault.argtypes = [i]
+    L.fa_test_set_fault.restype = None
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_tensor(name, t, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise RuntimeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _shapes(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, H, N, d]")
+    B, Hq, N, d = q.shape
+    return B, Hq, k.shape[1], N, d
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """Forward pass into caller-owned ``o`` [B,Hq,N,d] bf16 and ``lse`` [B,Hq,N] fp32."""
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    bf = torch.bfloat16
+    args = [_check_tensor("q", q, bf, (B, Hq, N, d)), _check_tensor("k", k, bf, (B, Hkv, N, d)),
+            _check_tensor("v", v, bf, (B, Hkv, N, d)), _check_tensor("o", o, bf, (B, Hq, N, d)),
+            _check_tensor("lse", lse, torch.float32, (B, Hq, N))]
+    rc = lib().fa_fwd(*args, B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+
+
+def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None) -> None:
+    """Backward pass into caller-owned ``dq``, ``dk``, ``dv`` using ``workspace`` (uint8 CUDA tensor)."""
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    bf = torch.bfloat16
+    args = [_check_tensor("q", q, bf, (B, Hq, N, d)), _check_tensor("k", k, bf, (B, Hkv, N, d)),
+            _check_tensor("v", v, bf, (B, Hkv, N, d)), _check_tensor("o", o, bf, (B, Hq, N, d)),
+            _check_tensor("dout", dout, bf, (B, Hq, N, d)),
+            _check_tensor("lse", lse, torch.float32, (B, Hq, N)),
+            _check_tensor("dq", dq, bf, (B, Hq, N, d)), _check_tensor("dk", dk, bf, (B, Hkv, N, d)),
+            _check_tensor("dv", dv, bf, (B, Hkv, N, d))]
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().fa_bwd(*args, B, Hq, Hkv, N, d, int(bool(causal)), float(scale), workspace.data_ptr(),
+                      ws_bytes, _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+
+
+def fa_check_device_error(stream=None) -> int:
+    return int(lib().fa_check_device_error(_stream(stream)))
+
+
+def fa_set_watchdog_ns(ns: int) -> None:
+    lib().fa_set_watchdog_ns(int(ns))
+
+
+def fa_test_set_fault(code: int) -> None:
+    lib().fa_test_set_fault(int(code))
+
+
+# ------------------------------------------------------------ conveniences
+
+def attention_forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
+    """Allocates ``o`` and ``lse`` with torch and runs :func:`fa_fwd`."""
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    scale = d ** -0.5 if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, dout, lse, causal: bool, scale: float | None = None, workspace=None,
+                       stream=None):
+    """Allocates ``dq``, ``dk``, ``dv`` (and the workspace if not given) and runs :func:`fa_bwd`."""
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    scale = d ** -0.5 if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_bytes(B, Hq, Hkv, N, d), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace, stream)
+    return dq, dk, dv

@@ -1,0 +1,121 @@
+/*
+ * fa.h - exact IO-aware attention for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * What is computed. For every batch b and query head h,
+ *     S = scale * Q K^T            (masked: S_ij = -inf for j > i when causal)
+ *     P = softmax(S) row by row,   O = P V,
+ *     L_i = log sum_j exp(S_ij)    (natural log, one fp32 per query row)
+ * which is the attention of "FlashAttention: IO-aware exact attention"
+ * (daily-term page, "NAIVE ATTENTION vs FLASHATTENTION" diagram, NAIVE box
+ * for the definition, FLASH box for the tiled online-softmax form and the
+ * per-row logsumexp it keeps). The forward never writes the N x N scores to
+ * memory; the backward rebuilds P from Q, K and L on chip (same page, "Four
+ * ideas" list, item "Recomputation in the backward pass").
+ * Grouped-query attention: query head h reads KV head h / (Hq / Hkv).
+ *
+ * Layout (all row-major, innermost dimension last, no padding):
+ *     q, o, dout, dq : bf16 [B][Hq][N][d]
+ *     k, v, dk, dv   : bf16 [B][Hkv][N][d]
+ *     lse            : fp32 [B][Hq][N]
+ * Supported: d in {64, 128}; Hq a multiple of Hkv; N >= 1; scale finite and
+ * > 0; every pointer 16-byte aligned; device of compute capability 10.0
+ * (B200, sm_100a).
+ *
+ * Ownership. Every pointer is device memory allocated and owned by the
+ * caller; the library never allocates or frees device memory and keeps no
+ * pointer after a call returns. Calls are asynchronous on `stream` (a
+ * cudaStream_t; NULL means the legacy default stream) and use the current
+ * CUDA device. Outputs are overwritten (dk and dv are not accumulated into).
+ *
+ * Errors. A nonzero status is returned before anything is launched when an
+ * argument is invalid (FA_ERR_INVALID_ARGUMENT) or a shape or device is not
+ * supported (FA_ERR_UNSUPPORTED); no output is touched in that case.
+ * FA_ERR_CUDA means a CUDA call failed while launching (the text of the CUDA
+ * error is available through fa_status_string until the next call on this
+ * thread). Every wait inside the kernels is bounded by a watchdog; a wait
+ * that runs out records a device error word instead of hanging, and
+ * fa_check_device_error reports it as FA_ERR_TIMEOUT.
+ *
+ * Thread safety: calls may be made from several host threads. The only
+ * shared state is a per-device cache of the device check and of the
+ * address of the error word.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA_OK 0
+#define FA_ERR_INVALID_ARGUMENT 1
+#define FA_ERR_UNSUPPORTED 2
+#define FA_ERR_CUDA 3
+#define FA_ERR_TIMEOUT 4
+
+/*
+ * Forward pass: o = softmax(scale * q k^T [causal]) v and lse = row
+ * logsumexp (natural log). Source: "FlashAttention: IO-aware exact
+ * attention", FLASH box of the "NAIVE ATTENTION vs FLASHATTENTION" diagram
+ * (tiled loop with running max m and sum l; O written once plus one
+ * logsumexp per row) and the "PREFILL PATH" diagram (128-row Q blocks,
+ * 128-column K/V blocks).
+ *   q [B][Hq][N][d], k, v [B][Hkv][N][d]  (bf16, read only)
+ *   o [B][Hq][N][d] (bf16, written), lse [B][Hq][N] (fp32, written)
+ *   causal: 0 or 1 (query i sees keys j <= i)
+ *   stream: cudaStream_t or NULL
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+           int d, int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for this shape: an fp32 row sum
+ * D_i = sum_c dout_ic o_ic per query row, and an fp32 dQ accumulator
+ * [B][Hq][N][d]. Returns 0 for an invalid or unsupported shape.
+ */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * Backward pass: gradients of sum(dout * o) with respect to q, k and v,
+ * rebuilding P from q, k and lse tile by tile. Source: "FlashAttention:
+ * IO-aware exact attention", "Four ideas" list, item "Recomputation in the
+ * backward pass" (only the per-row logsumexp is kept from the forward pass
+ * and P is rebuilt on chip); the gradient formulas are those of the
+ * definition above: dV = P^T dO, dP = dO V^T, D_i = sum_j P_ij dP_ij,
+ * dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q, with the query
+ * heads of a KV group summed into its dK, dV.
+ *   q, k, v, o, dout, lse: as produced for / by fa_fwd (read only)
+ *   dq [B][Hq][N][d], dk, dv [B][Hkv][N][d] (bf16, written)
+ *   workspace: device memory of at least fa_bwd_workspace_bytes(...) bytes,
+ *   16-byte aligned, owned by the caller, contents need not be initialised
+ *   and are clobbered. FA_ERR_INVALID_ARGUMENT if it is NULL or too small.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static text for a status code (for FA_ERR_CUDA: the last CUDA error seen by
+ * this thread). Never NULL. */
+const char* fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word. Returns FA_OK, FA_ERR_TIMEOUT when a kernel's bounded wait ran out
+ * since the last check, or FA_ERR_CUDA when the synchronisation failed.
+ */
+int fa_check_device_error(void* stream);
+
+/*
+ * Sets the per-wait watchdog budget in nanoseconds for later launches from
+ * any thread (default 2e9). Values below 1e6 are raised to 1e6.
+ */
+void fa_set_watchdog_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */
