@@ -1,17 +1,551 @@
-// Backward attention kernels for sm_100a (placeholder until the kernels land).
+// Backward attention kernels for sm_100a.
+//
+// Gradients of sum(dO * O) for O = softmax(scale * Q K^T [causal]) V, with P
+// rebuilt on chip from Q, K and the forward's row logsumexp L instead of
+// being stored (FlashAttention: IO-aware exact attention, "Four ideas" list,
+// item "Recomputation in the backward pass"; Flash Attention: memory-
+// efficient transformers, "Recomputation in the Backward Pass"). The pages
+// give no formulas; these are the gradient of the definition:
+//   P = exp(scale S - L), dV = P^T dO, dP = dO V^T, D_i = sum_j P_ij dP_ij
+//   (= sum_c dO_ic O_ic), dS = P o (dP - D), dQ = scale dS K,
+//   dK = scale dS^T Q, KV heads summing over their query heads.
+//
+// Three kernels:
+//   bwd_pre   D_i = sum_c dO_ic O_ic (fp32) and zero the fp32 dQ accumulator.
+//   bwd_main  one CTA per (batch, KV head, 128-key tile j). K_j and V_j stay in
+//             shared memory; the CTA loops over the query heads of the KV
+//             group and the 128-row query tiles i that can see tile j
+//             (i >= j when causal). Per (head, i):
+//               S^T  = K_j Q_i^T          (tcgen05 -> tensor memory)
+//               dP^T = V_j dO_i^T         (tcgen05 -> tensor memory)
+//               P^T  = 2^(S^T scale log2e - L_i log2e), dS^T = P^T o (dP^T - D_i)
+//                                         (one thread per key row)
+//               dV_j += P^T dO_i          (P^T read from tensor memory)
+//               dK_j += dS^T Q_i          (dS^T from shared memory)
+//               dQ_i  = dS K_j            (same dS^T bytes read MN-major)
+//             and dQ_i is added to the fp32 accumulator with vector
+//             reductions. dK_j (times scale) and dV_j are written once.
+//   bwd_post  dq = bf16(scale * accumulator).
+//
+// Warp roles of bwd_main (384 threads):
+//   warps 0-3   softmax-gradient warpgroup: thread = key row; writes P^T to
+//               tensor memory and dS^T to shared memory; epilogue stores dV.
+//   warps 4-7   dQ warpgroup: thread = query row; reads dQ_i out of tensor
+//               memory and reduces it into the accumulator; epilogue stores dK.
+//   warp 8      producer: K_j, V_j once; Q_i, dO_i by TMA and L_i, D_i by
+//               plain loads into a two-stage ring.
+//   warp 9      tensor-memory owner and MMA issuer.
+// Tensor memory: [0,128) S^T | [128,256) dP^T, then P^T (bf16) in its first
+// 64 columns, then dQ_i | dV_j (D columns) | dK_j (D columns).
+// Every tcgen05 operation of the MMA thread completes in issue order, which
+// orders P^T reads before the dQ write into the same columns.
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
 #include "fa_internal.h"
+#include "sm100.cuh"
 
 namespace fa {
+namespace {
+
+constexpr int kB = 128;  // rows per Q tile and per K/V tile
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kBoxBytes = kB * 64 * 2;
+  static constexpr int kTileBytes = kBoxBytes * (D / 64);  // one 128 x D bf16 tile
+  static constexpr int kStages = 2;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;                  // [stage] Q_i
+  static constexpr int kOffDO = kOffQ + kStages * kTileBytes;       // [stage] dO_i
+  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;      // dS^T, 128 x 128 bf16
+  static constexpr int kOffLD = kOffDS + 2 * kBoxBytes;             // [stage] L2[128], D[128]
+  static constexpr int kOffBar = kOffLD + kStages * 2 * kB * 4;
+  static constexpr int kUsed = kOffBar + 256;
+  static constexpr int kSmemBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static_assert(kUsed <= 232448, "shared memory budget");
+  static_assert(kSmemBytes > 114 * 1024, "one CTA per SM (owns all tensor memory)");
+};
+
+struct BwdArgs {
+  const float* lse;
+  const float* dsum;    // D_i, fp32 [B*Hq*N]
+  float* dq_acc;        // fp32 [B*Hq*N*d]
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int N, Hq, Hkv, BHkv, nk, nq;
+  float scale, scale_log2;
+  LaunchCtl ctl;
+};
+
+struct BwdBars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full, dp_full, p_ready, ds_free, dq_full, dq_empty, acc_final, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdArgs a) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+  if (pad + C::kUsed > static_cast<uint32_t>(C::kSmemBytes)) {
+    // Not enough room to align the tiles: report instead of overrunning.
+    if (threadIdx.x == 0) atomicOr(a.ctl.err, 2u);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::kOffBar);
+  float* sLD = reinterpret_cast<float*>(smem + C::kOffLD);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // Work unit: (batch, KV head, key tile j); the longest units (smallest j
+  // when causal) get the lowest block indices.
+  const int bkv = blockIdx.x % a.BHkv;
+  const int j = blockIdx.x / a.BHkv;
+  const int r = a.Hq / a.Hkv;
+  const int b = bkv / a.Hkv;
+  const int g = bkv % a.Hkv;
+  const int i0 = CAUSAL ? j : 0;
+  const int nqi = a.nq - i0;     // query tiles per head
+  const int n_it = r * nqi;      // (head, query tile) iterations
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->p_ready, kB);
+    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, kB);
+    mbar_init(&bars->acc_final, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const Watch w{&bars->abort, a.ctl.err, a.ctl.budget_ns};
+
+  const uint32_t sK = smem_u32(smem + C::kOffK);
+  const uint32_t sV = smem_u32(smem + C::kOffV);
+  const uint32_t sQ = smem_u32(smem + C::kOffQ);
+  const uint32_t sDO = smem_u32(smem + C::kOffDO);
+  const uint32_t sDS = smem_u32(smem + C::kOffDS);
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    int q_last[2] = {-1, -1};
+    bool kv_issued = false;
+    bool ok = true;
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_3d(&tmK, &bars->kv_full, smem + C::kOffK + x * C::kBoxBytes, x * 64, j * kB, bkv);
+        tma_load_3d(&tmV, &bars->kv_full, smem + C::kOffV + x * C::kBoxBytes, x * 64, j * kB, bkv);
+      }
+      kv_issued = true;
+    }
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it & 1;
+      const int u = it >> 1;
+      if (it >= 2) {
+        ok = __all_sync(0xffffffffu, wait_bar(&bars->q_empty[s], (u - 1) & 1, w));
+        if (!ok) break;
+      }
+      const int h = g * r + it / nqi;
+      const int i = i0 + it % nqi;
+      const int bh = b * a.Hq + h;
+      // L (in log2 units) and D for the 128 query rows of this tile; rows
+      // past N get L = +inf so that their P is exactly 0.
+      float* l2 = sLD + s * 2 * kB;
+      float* dd = l2 + kB;
+#pragma unroll
+      for (int e = 0; e < kB / 32; ++e) {
+        const int rr = e * 32 + lane;
+        const int row = i * kB + rr;
+        const bool in = row < a.N;
+        const size_t idx = static_cast<size_t>(bh) * a.N + row;
+        l2[rr] = in ? a.lse[idx] * kLog2e : CUDART_INF_F;
+        dd[rr] = in ? a.dsum[idx] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::kTileBytes);
+        for (int x = 0; x < D / 64; ++x) {
+          tma_load_3d(&tmQ, &bars->q_full[s], smem + C::kOffQ + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                      i * kB, bh);
+          tma_load_3d(&tmDO, &bars->q_full[s], smem + C::kOffDO + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                      i * kB, bh);
+        }
+        q_last[s] = u;
+      }
+    }
+    if (lane == 0) {
+      if (kv_issued) drain_bar(&bars->kv_full, 0, w);
+      for (int s = 0; s < 2; ++s)
+        if (q_last[s] >= 0) drain_bar(&bars->q_full[s], q_last[s] & 1, w);
+    }
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t id_sdp = idesc_bf16(kB, kB, false, false);  // S^T, dP^T
+      constexpr uint32_t id_dv = idesc_bf16(kB, D, false, true);     // dV (A in tensor memory)
+      constexpr uint32_t id_dk = idesc_bf16(kB, D, false, true);     // dK
+      constexpr uint32_t id_dq = idesc_bf16(kB, D, true, true);      // dQ (A = dS, MN-major)
+      const uint32_t tS = tmem + C::kColS, tDP = tmem + C::kColDP;
+      const uint32_t tDV = tmem + C::kColDV, tDK = tmem + C::kColDK;
+      auto kdesc = [](uint32_t base, int k) {  // K-major operand, K step k (16 elements)
+        return sdesc_sw128(base + (k / 4) * (kB * 128) + (k % 4) * 32, 16, 1024);
+      };
+      auto mdesc = [](uint32_t base, int k) {  // MN-major operand, K step k (16 rows)
+        return sdesc_sw128(base + k * 2048, kB * 128, 1024);
+      };
+      auto issue_sdp = [&](int s) {
+        const uint32_t q = sQ + s * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) mma_ss(tS, kdesc(sK, k), kdesc(q, k), id_sdp, k > 0);
+        mma_commit(&bars->s_full);
+      };
+      auto issue_dp = [&](int s) {
+        const uint32_t o = sDO + s * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(sV, k), kdesc(o, k), id_sdp, k > 0);
+        mma_commit(&bars->dp_full);
+      };
+      bool ok = wait_bar(&bars->kv_full, 0, w) && wait_bar(&bars->q_full[0], 0, w);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0);
+        issue_dp(0);
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it & 1;
+        if (!(ok = wait_bar(&bars->p_ready, it & 1, w))) break;
+        tc_fence_after();
+        const uint32_t q = sQ + s * C::kTileBytes, o = sDO + s * C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < kB / 16; ++k) mma_ts(tDV, tDP + k * 8, mdesc(o, k), id_dv, (it > 0 || k > 0));
+#pragma unroll
+        for (int k = 0; k < kB / 16; ++k) mma_ss(tDK, kdesc(sDS, k), mdesc(q, k), id_dk, (it > 0 || k > 0));
+#pragma unroll
+        for (int k = 0; k < kB / 16; ++k) mma_ss(tDP, mdesc(sDS, k), mdesc(sK, k), id_dq, k > 0);
+        mma_commit(&bars->dq_full);
+        mma_commit(&bars->ds_free);
+        mma_commit(&bars->q_empty[s]);
+        if (it + 1 < n_it) {
+          const int s1 = (it + 1) & 1;
+          if (!(ok = wait_bar(&bars->q_full[s1], ((it + 1) >> 1) & 1, w))) break;
+          tc_fence_after();
+          issue_sdp(s1);
+          if (!(ok = wait_bar(&bars->dq_empty, it & 1, w))) break;
+          tc_fence_after();
+          issue_dp(s1);
+        }
+      }
+      mma_commit(&bars->acc_final);
+      mma_commit(&bars->drain);
+      drain_bar(&bars->drain, 0, w);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------- P^T and dS^T (key rows)
+    const int quad = warp & 3;
+    const int kr = quad * 32 + lane;                       // key row in tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS;
+    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const float sl2 = a.scale_log2;
+    uint8_t* ds_row = smem + C::kOffDS + kr * 128;         // row kr of both 64-column boxes
+    const uint32_t sw = static_cast<uint32_t>(kr & 7);
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it & 1;
+      const int i = i0 + it % nqi;
+      const float* l2 = sLD + s * 2 * kB;
+      const float* dd = l2 + kB;
+      // q_full orders the producer's plain stores of L and D before these reads.
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[s], (it >> 1) & 1, w));
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full, it & 1, w));
+      if (ok && it > 0) ok = __all_sync(0xffffffffu, wait_bar(&bars->ds_free, (it - 1) & 1, w));
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->dp_full, it & 1, w));
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = CAUSAL && (i == j);
+#pragma unroll
+      for (int c = 0; c < kB / 32; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_ld32(tDP + c * 32, dv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q0 = c * 32 + 2 * e;
+          float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l2[q0]));
+          float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l2[q0 + 1]));
+          if (diag) {
+            if (q0 < kr) p0 = 0.f;
+            if (q0 + 1 < kr) p1 = 0.f;
+          }
+          const float d0 = p0 * (__uint_as_float(dv[2 * e]) - dd[q0]);
+          const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - dd[q0 + 1]);
+          pk[e] = pack_bf16x2(p0, p1);
+          dk[e] = pack_bf16x2(d0, d1);
+        }
+        // P^T chunk -> tensor memory columns [16c, 16c+16) of the dP^T block
+        // (those columns' dP^T values were consumed by this or an earlier chunk).
+        tmem_st16(tDP + c * 16, pk);
+        // dS^T chunk: queries [32c, 32c+32) of key row kr, 128-byte swizzled.
+        uint8_t* box = ds_row + (c >> 1) * (kB * 128);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t chunk = static_cast<uint32_t>((c & 1) * 4 + u);
+          uint4 val = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          *reinterpret_cast<uint4*>(box + ((chunk ^ sw) << 4)) = val;
+        }
+      }
+      tmem_st_wait();
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->p_ready);
+    }
+    // Epilogue: dV_j rows (this thread's key row).
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
+    if (ok) {
+      tc_fence_after();
+      const int key = j * kB + kr;
+      __nv_bfloat16* dst = a.dv + (static_cast<size_t>(bkv) * a.N + key) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t vv[32];
+        tmem_ld32(tmem + lane_off + C::kColDV + c * 32, vv);
+        uint4 o4[4];
+        uint32_t* po = reinterpret_cast<uint32_t*>(o4);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) po[e] = pack_bf16x2(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1]));
+        if (key < a.N) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(dst + c * 32)[e] = o4[e];
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ----------------------------------------------- dQ_i readout (query rows)
+    const int quad = warp & 3;
+    const int qr = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tDQ = tmem + lane_off + C::kColDP;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->dq_full, it & 1, w));
+      if (!ok) break;
+      tc_fence_after();
+      const int h = g * r + it / nqi;
+      const int i = i0 + it % nqi;
+      const int row = i * kB + qr;
+      float* dst = a.dq_acc + ((static_cast<size_t>(b) * a.Hq + h) * a.N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t vv[32];
+        tmem_ld32(tDQ + c * 32, vv);
+        if (row < a.N) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(vv[4 * e]), __uint_as_float(vv[4 * e + 1]),
+                       __uint_as_float(vv[4 * e + 2]), __uint_as_float(vv[4 * e + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+    }
+    // Epilogue: dK_j = scale * accumulated dS^T Q (this thread's key row).
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
+    if (ok) {
+      tc_fence_after();
+      const int key = j * kB + qr;
+      __nv_bfloat16* dst = a.dk + (static_cast<size_t>(bkv) * a.N + key) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t vv[32];
+        tmem_ld32(tmem + lane_off + C::kColDK + c * 32, vv);
+        uint4 o4[4];
+        uint32_t* po = reinterpret_cast<uint32_t*>(o4);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          po[e] = pack_bf16x2(__uint_as_float(vv[2 * e]) * a.scale, __uint_as_float(vv[2 * e + 1]) * a.scale);
+        if (key < a.N) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(dst + c * 32)[e] = o4[e];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// D_i = sum_c dO_ic O_ic for every query row, and zero the dQ accumulator.
+// One warp per row; each lane handles 8 columns per step (one uint4 each).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ dout,
+                                                      float* __restrict__ dsum, float* __restrict__ dq_acc,
+                                                      long long rows) {
+  const long long warp_g = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long row = warp_g; row < rows; row += nwarps) {
+    float acc = 0.f;
+    if (lane * 8 < D) {
+      const uint4 a4 = reinterpret_cast<const uint4*>(o + row * D)[lane];
+      const uint4 b4 = reinterpret_cast<const uint4*>(dout + row * D)[lane];
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a4);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b4);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(a2[e]);
+        const float2 fb = __bfloat1622float2(b2[e]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) dsum[row] = acc;
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
+    for (int e = lane; e < D / 4; e += 32) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// dq = bf16(scale * accumulator), 8 elements per thread per step.
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ dq_acc,
+                                                       __nv_bfloat16* __restrict__ dq, float scale,
+                                                       long long n8) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n8; e += stride) {
+    const float4 x = reinterpret_cast<const float4*>(dq_acc)[2 * e];
+    const float4 y = reinterpret_cast<const float4*>(dq_acc)[2 * e + 1];
+    uint4 out;
+    out.x = pack_bf16x2(x.x * scale, x.y * scale);
+    out.y = pack_bf16x2(x.z * scale, x.w * scale);
+    out.z = pack_bf16x2(y.x * scale, y.y * scale);
+    out.w = pack_bf16x2(y.z * scale, y.w * scale);
+    reinterpret_cast<uint4*>(dq)[e] = out;
+  }
+}
+
+int grid_for(long long work, int per_block, int cap) {
+  long long g = (work + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  return static_cast<int>(g < cap ? g : cap);
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const void* o, const void* dout, const float* lse, void* dq,
+                         void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  const long long rows = static_cast<long long>(s.B) * s.Hq * s.N;
+  float* dsum = static_cast<float*>(workspace);
+  const size_t dsum_bytes = ((static_cast<size_t>(rows) * 4 + 255) / 256) * 256;
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsum_bytes);
+
+  bwd_pre_kernel<D><<<grid_for(rows, 8, 148 * 64), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  auto kern = bwd_main_kernel<D, CAUSAL>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  BwdArgs a;
+  a.lse = lse;
+  a.dsum = dsum;
+  a.dq_acc = dq_acc;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.N = s.N;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.BHkv = s.B * s.Hkv;
+  a.nk = (s.N + kB - 1) / kB;
+  a.nq = a.nk;
+  a.scale = s.scale;
+  a.scale_log2 = s.scale * kLog2e;
+  a.ctl = ctl;
+  const long long grid = static_cast<long long>(a.nk) * a.BHkv;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  const long long n8 = rows * D / 8;
+  bwd_post_kernel<<<grid_for(n8, 256, 148 * 32), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                                     s.scale, n8);
+  return cudaGetLastError();
+}
+
+}  // namespace
 
 size_t bwd_workspace_bytes(const AttnShape& s) {
   const size_t rows = static_cast<size_t>(s.B) * s.Hq * s.N;
-  return rows * 4 + rows * s.d * 4 + 256;
+  const size_t dsum_bytes = ((rows * 4 + 255) / 256) * 256;
+  return dsum_bytes + rows * static_cast<size_t>(s.d) * 4;
 }
 
-cudaError_t launch_bwd(const AttnShape&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                       const CUtensorMap&, const void*, const void*, const float*, void*, void*, void*, void*,
-                       const LaunchCtl&, cudaStream_t) {
-  return cudaErrorNotYetImplemented;
+cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const void* o, const void* dout, const float* lse, void* dq,
+                       void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream) {
+  if (s.d == 64)
+    return s.causal ? launch_bwd_t<64, true>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream)
+                    : launch_bwd_t<64, false>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream);
+  return s.causal ? launch_bwd_t<128, true>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream)
+                  : launch_bwd_t<128, false>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream);
 }
 
 }  // namespace fa
