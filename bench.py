@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the attention hot path: one step = forward +
+backward of one batch of the workload (default: B=2, H=16, N=8192, d=128,
+causal, Q and K drawn with gain 2), inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+    python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
+
+Prints one JSON line (rank 0). Multi-GPU runs are weak scaling: every rank
+runs its own batch of the same per-GPU size (attention over independent
+(batch, head) slices needs no exchange), timed on the device between
+barriers, maximum over ranks. FLOPs are algorithmic: 4*B*Hq*N^2*d for the
+forward (half when causal) and 2.5x that for the backward.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16) and fraction of B200 dense BF16 peak"
+DEFAULT_WORKLOAD = "fwdbwd_b2_h16_n8192_d128_causal_peaky"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(
+        os.environ.get("LOCAL_RANK", "0"))
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity without a group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w, seconds: float, max_slices: int = 64):
+    """Times the fp64 oracle (as it stands) on whole (batch, head) slices of
+    the workload until about ``seconds`` have passed. Returns
+    (algorithmic FLOPs done, wall seconds, slices, threads)."""
+    import oracle
+    from exact_io_aware_56_b200 import make_inputs, to_f64
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover - threadpoolctl missing
+        threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    flops_slice = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.Hq)
+    done, elapsed, n = 0.0, 0.0, 0
+    while n < max_slices and (elapsed < seconds or n == 0):
+        host = make_inputs(1, 1, 1, w.N, w.d, w.seed + 7919 * (n + 1), w.qk_gain, w.backward)
+        ref = {k: to_f64(v) for k, v in host.items()}
+        t0 = time.perf_counter()
+        oracle.attn_fwd_ref(ref["q"], ref["k"], ref["v"], w.causal, w.scale)
+        if w.backward:
+            oracle.attn_bwd_ref(ref["q"], ref["k"], ref["v"], ref["dout"], w.causal, w.scale)
+        elapsed += time.perf_counter() - t0
+        done += flops_slice
+        n += 1
+    return done, elapsed, n, threads
+
+
+def reference_arm(args):
+    from exact_io_aware_56_b200 import WORKLOADS
+
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    times = []
+    flops_slice = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.Hq)
+    threads = 1
+    for it in range(args.warmup + args.steps):
+        _, el, _, threads = oracle_sample(w, 0.0, max_slices=1)
+        if it >= args.warmup:
+            times.append(el)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops_slice / (ms * 1e-3) / 1e12
+    sample = f"one (batch, head) slice of {w.name} (fwd+bwd, fp64 oracle) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ native arm
+
+def native_arm(args):
+    import torch
+
+    from exact_io_aware_56_b200 import WORKLOADS, fa, make_inputs
+
+    w = WORKLOADS[args.workload]
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device; there is no CPU path")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl")
+    fa.lib()
+
+    host = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + rank, w.qk_gain, w.backward)
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    dout = host["dout"].to(dev) if w.backward else None
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    o_resid = None
+    if w.backward:
+        # Training path: the forward also keeps o's rounding residual for D.
+        o_resid = torch.empty_like(q)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.fa_fwd(q, k, v, o, lse, w.causal, w.scale, stream, o_resid=o_resid)
+        if ev is not None:
+            ev[1].record(stream)
+        if w.backward:
+            fa.fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, w.causal, w.scale, ws, stream, o_resid=o_resid)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_check_device_error(stream) != fa.FA_OK:
+        raise RuntimeError("device watchdog fired during warm-up")
+
+    # Per-step events: [fwd start, fwd end, bwd pre end, bwd main end, step end].
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for e in evs:  # torch creates the CUDA event on first record; the hook needs real handles
+        e[2].record(stream)
+        e[3].record(stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        t_start.record(stream)
+        for s in range(args.steps):
+            if w.backward:
+                fa.fa_profile_set_bwd_events(evs[s][2], evs[s][3])
+            step(evs[s])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    fa.fa_profile_set_bwd_events(None, None)
+    barrier(dev)
+    if fa.fa_check_device_error(stream) != fa.FA_OK:
+        raise RuntimeError("device watchdog fired during the timed steps")
+    ms_local = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(ms_local, dev)
+    step_flops = w.fwd_flops() + w.bwd_flops()
+    value = step_flops * args.steps * world / (ms_total * 1e-3) / 1e12
+
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    kernels = {"fwd": {"ms": fwd_ms, "flops": w.fwd_flops(), "launches_per_step": 1}}
+    if w.backward:
+        kernels["bwd_main"] = {"ms": statistics.mean(e[2].elapsed_time(e[3]) for e in evs),
+                               "flops": w.bwd_flops(), "launches_per_step": 1}
+        kernels["bwd_pre"] = {"ms": statistics.mean(e[1].elapsed_time(e[2]) for e in evs)}
+        kernels["bwd_post"] = {"ms": statistics.mean(e[3].elapsed_time(e[4]) for e in evs)}
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    for kn in ("fwd", "bwd_main"):
+        if kn in kernels:
+            kk = kernels[kn]
+            kk["tflops"] = kk["flops"] / (kk["ms"] * 1e-3) / 1e12
+            kk["frac"] = kk["tflops"] / peak
+    dom = max((kn for kn in ("fwd", "bwd_main") if kn in kernels), key=lambda kn: kernels[kn]["ms"])
+    roofline = {
+        "bound": "tensor", "kernel": dom, "achieved": kernels[dom]["tflops"], "peak": peak, "unit": "TFLOP/s",
+        "frac": kernels[dom]["frac"], "traffic": None,
+        "peak_source": f"{peak_src} bf16 dense (burst)",
+        "kernels": {kn: {x: kernels[kn][x] for x in ("ms", "tflops", "frac") if x in kernels[kn]}
+                    for kn in kernels},
+    }
+
+    # End to end through the public API: pinned host inputs copied in, both
+    # passes run, every output copied back, all inside the timed region.
+    e2e = None
+    if args.e2e_steps > 0:
+        hin = {n: host[n].pin_memory() for n in host}
+        outs = [o, lse] + ([dq, dk, dv] if w.backward else [])
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        dins = {"q": q, "k": k, "v": v}
+        if w.backward:
+            dins["dout"] = dout
+
+        def e2e_step():
+            for n, t in dins.items():
+                t.copy_(hin[n], non_blocking=True)
+            step()
+            for src, dst in zip(outs, hout):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": step_flops * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops, secs, n, threads = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} whole (batch, head) slices of {w.name}, fwd+bwd, fp64 oracle, {secs:.1f} s"}
+
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v) + ((dout,) if w.backward else ()))
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "qk_gain": w.qk_gain, "global_batch": w.B * world,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per rank), no flush"},
+        "fraction_of_peak": value / world / peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * (4 if w.backward else 1),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference_arm(args)
+    return native_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -8,6 +8,8 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "../../include/fa_profile.h"
+#include "../../include/fa_test.h"
 #include "fa_internal.h"
 
 namespace fa {
@@ -20,6 +22,8 @@ __device__ unsigned int g_err_word;
 
 std::atomic<uint64_t> g_budget_ns{2000000000ull};
 std::atomic<int> g_fault{0};
+std::atomic<void*> g_ev_pre{nullptr};
+std::atomic<void*> g_ev_main{nullptr};
 thread_local char t_cuda_msg[256] = "no CUDA error recorded";
 
 struct DevState {
@@ -84,6 +88,8 @@ LaunchCtl make_ctl(const DevState* st) {
   c.err = st->err;
   c.budget_ns = g_budget_ns.load(std::memory_order_relaxed);
   c.fault = g_fault.load(std::memory_order_relaxed);
+  c.ev_after_pre = static_cast<cudaEvent_t>(g_ev_pre.load(std::memory_order_relaxed));
+  c.ev_after_main = static_cast<cudaEvent_t>(g_ev_main.load(std::memory_order_relaxed));
   return c;
 }
 
@@ -115,10 +121,11 @@ using namespace fa;
 
 extern "C" {
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
-           int d, int causal, float scale, void* stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse, int B,
+                    int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(o_resid))
     return FA_ERR_INVALID_ARGUMENT;
   int rc = check_shape(B, Hq, Hkv, N, d, causal, scale);
   if (rc != FA_OK) return rc;
@@ -129,8 +136,19 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
       !encode_tile_map(&tv, v, d, N, B * Hkv, 128))
     return FA_ERR_UNSUPPORTED;
   AttnShape s{B, Hq, Hkv, N, d, causal, scale};
-  cudaError_t e = launch_fwd(s, tq, tk, tv, o, lse, make_ctl(st), static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_fwd(s, tq, tk, tv, o, o_resid, lse, make_ctl(st), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+           int d, int causal, float scale, void* stream) {
+  return fwd_impl(q, k, v, o, nullptr, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+}
+
+int fa_fwd_with_residual(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse, int B,
+                         int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  if (!o_resid) return FA_ERR_INVALID_ARGUMENT;
+  return fwd_impl(q, k, v, o, o_resid, lse, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
@@ -139,11 +157,11 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   return bwd_workspace_bytes(s);
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-           void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
-           void* workspace, size_t workspace_bytes, void* stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                    const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                    int d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARGUMENT;
-  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+  const void* ptrs[] = {q, k, v, o, o_resid, dout, lse, dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return FA_ERR_INVALID_ARGUMENT;
   int rc = check_shape(B, Hq, Hkv, N, d, causal, scale);
@@ -156,9 +174,25 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
   if (!encode_tile_map(&tq, q, d, N, B * Hq, 128) || !encode_tile_map(&tk, k, d, N, B * Hkv, 128) ||
       !encode_tile_map(&tv, v, d, N, B * Hkv, 128) || !encode_tile_map(&tdo, dout, d, N, B * Hq, 128))
     return FA_ERR_UNSUPPORTED;
-  cudaError_t e = launch_bwd(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, make_ctl(st),
+  cudaError_t e = launch_bwd(s, tq, tk, tv, tdo, o, o_resid, dout, lse, dq, dk, dv, workspace, make_ctl(st),
                              static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+           void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, nullptr, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, workspace,
+                  workspace_bytes, stream);
+}
+
+int fa_bwd_with_residual(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                         int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (!o_resid) return FA_ERR_INVALID_ARGUMENT;
+  return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, workspace,
+                  workspace_bytes, stream);
 }
 
 const char* fa_status_string(int status) {
@@ -203,5 +237,10 @@ void fa_set_watchdog_ns(uint64_t ns) { g_budget_ns.store(ns < 1000000ull ? 10000
 // (1 = the forward producer never loads the first K tile) so that the
 // watchdog path can be exercised without faulting the GPU.
 void fa_test_set_fault(int code) { g_fault.store(code); }
+
+void fa_profile_set_bwd_events(void* after_pre, void* after_main) {
+  g_ev_pre.store(after_pre);
+  g_ev_main.store(after_main);
+}
 
 }  // extern "C"

@@ -12,6 +12,9 @@
 //
 // Three kernels:
 //   bwd_pre   D_i = sum_c dO_ic O_ic (fp32) and zero the fp32 dQ accumulator.
+//             O is the bf16 o plus, when given, its rounding residual: D_i
+//             multiplies every error of O by dO and sums it over d, and the
+//             bf16 rounding of O alone moves D by ~1e-2 at d = 128.
 //   bwd_main  one CTA per (batch, KV head, 128-key tile j). K_j and V_j stay in
 //             shared memory; the CTA loops over the query heads of the KV
 //             group and the 128-row query tiles i that can see tile j
@@ -433,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One warp per row; each lane handles 8 columns per step (one uint4 each).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ o_resid,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       float* __restrict__ dsum, float* __restrict__ dq_acc,
                                                       long long rows) {
@@ -444,14 +448,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
     if (lane * 8 < D) {
       const uint4 a4 = reinterpret_cast<const uint4*>(o + row * D)[lane];
       const uint4 b4 = reinterpret_cast<const uint4*>(dout + row * D)[lane];
+      const uint4 r4 = o_resid ? reinterpret_cast<const uint4*>(o_resid + row * D)[lane] : make_uint4(0, 0, 0, 0);
       const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a4);
       const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b4);
+      const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&r4);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 fa = __bfloat1622float2(a2[e]);
+        const float2 fr = __bfloat1622float2(r2[e]);
         const float2 fb = __bfloat1622float2(b2[e]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
+        acc = fmaf(fa.x + fr.x, fb.x, acc);
+        acc = fmaf(fa.y + fr.y, fb.y, acc);
       }
     }
 #pragma unroll
@@ -487,8 +494,9 @@ int grid_for(long long work, int per_block, int cap) {
 
 template <int D, bool CAUSAL>
 cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const void* o, const void* dout, const float* lse, void* dq,
-                         void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream) {
+                         const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
+                         cudaStream_t stream) {
   using C = BwdCfg<D>;
   const long long rows = static_cast<long long>(s.B) * s.Hq * s.N;
   float* dsum = static_cast<float*>(workspace);
@@ -496,9 +504,11 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsum_bytes);
 
   bwd_pre_kernel<D><<<grid_for(rows, 8, 148 * 64), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc, rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_resid),
+      static_cast<const __nv_bfloat16*>(dout), dsum, dq_acc, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (ctl.ev_after_pre && (e = cudaEventRecord(ctl.ev_after_pre, stream)) != cudaSuccess) return e;
 
   auto kern = bwd_main_kernel<D, CAUSAL>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -523,6 +533,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (ctl.ev_after_main && (e = cudaEventRecord(ctl.ev_after_main, stream)) != cudaSuccess) return e;
 
   const long long n8 = rows * D / 8;
   bwd_post_kernel<<<grid_for(n8, 256, 148 * 32), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
@@ -539,13 +550,13 @@ size_t bwd_workspace_bytes(const AttnShape& s) {
 }
 
 cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const void* o, const void* dout, const float* lse, void* dq,
-                       void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream) {
-  if (s.d == 64)
-    return s.causal ? launch_bwd_t<64, true>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream)
-                    : launch_bwd_t<64, false>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream);
-  return s.causal ? launch_bwd_t<128, true>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream)
-                  : launch_bwd_t<128, false>(s, tq, tk, tv, tdo, o, dout, lse, dq, dk, dv, workspace, ctl, stream);
+                       const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
+                       cudaStream_t stream) {
+#define FA_BWD_ARGS s, tq, tk, tv, tdo, o, o_resid, dout, lse, dq, dk, dv, workspace, ctl, stream
+  if (s.d == 64) return s.causal ? launch_bwd_t<64, true>(FA_BWD_ARGS) : launch_bwd_t<64, false>(FA_BWD_ARGS);
+  return s.causal ? launch_bwd_t<128, true>(FA_BWD_ARGS) : launch_bwd_t<128, false>(FA_BWD_ARGS);
+#undef FA_BWD_ARGS
 }
 
 }  // namespace fa

@@ -33,9 +33,8 @@
 // until P_t^(j+1) is handed back.
 //
 // The exponentials are base 2: scores are scaled by scale*log2(e), and
-// L = (m + log2 l) * ln 2. The rescale of O is lazy: a warp rescales only
-// when some row's max grew by more than 8 (a factor 256), otherwise every
-// row keeps its stale max, which changes no result because l and O share it.
+// L = (m + log2 l) * ln 2. A warp whose rows' maxima did not grow on a tile
+// skips the tensor-memory round trip of the O rescale.
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -51,7 +50,12 @@ constexpr int kBN = 128;   // keys per K/V tile
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// A warp rescales its O rows whenever some row's running max grew. Keeping
+// every row's reference max exact makes the largest weight of a row exactly
+// 1, which bf16 represents without error; a stale reference (deferring the
+// rescale until the max grew by more than a margin) turns that weight into
+// 2^delta, whose bf16 rounding moves O by up to 2^-9 |V| on peaky rows.
+constexpr float kRescaleThreshold = 0.0f;  // log2 units
 
 template <int D>
 struct FwdCfg {
@@ -72,6 +76,7 @@ struct FwdCfg {
 
 struct FwdArgs {
   __nv_bfloat16* o;
+  __nv_bfloat16* o_resid;  // optional: bf16(O - bf16(O)), the rounding residual of o
   float* lse;
   int N, Hq, Hkv, BH, n_pairs, nk;
   float scale_log2;
@@ -324,19 +329,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.N + row) * D;
+      __nv_bfloat16* rrow = a.o_resid ? a.o_resid + (static_cast<size_t>(bh) * a.N + row) * D : nullptr;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t oo[32];
         tmem_ld32(tO + c * 32, oo);
-        uint4 v[4];
+        uint4 v[4], res[4];
         uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+        uint32_t* pr = reinterpret_cast<uint32_t*>(res);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pv[i] = pack_bf16x2(__uint_as_float(oo[2 * i]) * inv_l, __uint_as_float(oo[2 * i + 1]) * inv_l);
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = __uint_as_float(oo[2 * i]) * inv_l;
+          const float x1 = __uint_as_float(oo[2 * i + 1]) * inv_l;
+          pv[i] = pack_bf16x2(x0, x1);
+          const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pv[i]);
+          pr[i] = pack_bf16x2(x0 - __low2float(hi), x1 - __high2float(hi));
+        }
         if (row < a.N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = v[i];
+          if (rrow) {
+            uint4* rd = reinterpret_cast<uint4*>(rrow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rd[i] = res[i];
+          }
         }
       }
       if (row < a.N) a.lse[static_cast<size_t>(bh) * a.N + row] = (m + lg2(l)) * 0.69314718055994530942f;
@@ -354,13 +371,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool CAUSAL>
 cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         void* o, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
+                         void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
   using C = FwdCfg<D>;
   auto kern = fwd_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
+  a.o_resid = static_cast<__nv_bfloat16*>(o_resid);
   a.lse = lse;
   a.N = s.N;
   a.Hq = s.Hq;
@@ -379,12 +397,12 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
 }  // namespace
 
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       void* o, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
+                       void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
   if (s.d == 64)
-    return s.causal ? launch_fwd_t<64, true>(s, tq, tk, tv, o, lse, ctl, stream)
-                    : launch_fwd_t<64, false>(s, tq, tk, tv, o, lse, ctl, stream);
-  return s.causal ? launch_fwd_t<128, true>(s, tq, tk, tv, o, lse, ctl, stream)
-                  : launch_fwd_t<128, false>(s, tq, tk, tv, o, lse, ctl, stream);
+    return s.causal ? launch_fwd_t<64, true>(s, tq, tk, tv, o, o_resid, lse, ctl, stream)
+                    : launch_fwd_t<64, false>(s, tq, tk, tv, o, o_resid, lse, ctl, stream);
+  return s.causal ? launch_fwd_t<128, true>(s, tq, tk, tv, o, o_resid, lse, ctl, stream)
+                  : launch_fwd_t<128, false>(s, tq, tk, tv, o, o_resid, lse, ctl, stream);
 }
 
 }  // namespace fa

@@ -19,19 +19,23 @@ struct LaunchCtl {
   unsigned int* err;        // device error word (watchdog)
   uint64_t budget_ns;       // watchdog budget per wait
   int fault;                // test-only fault injection selector (0 = none)
+  cudaEvent_t ev_after_pre;   // optional timing events (see fa_profile.h)
+  cudaEvent_t ev_after_main;
 };
 
 // Encodes a 3-D bf16 tensor map over [outer][rows][cols] with a box of
 // 64 columns x box_rows rows and 128-byte swizzle. Returns false on failure.
 bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows);
 
+// o_resid may be null (no residual written).
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       void* o, float* lse, const LaunchCtl& ctl, cudaStream_t stream);
+                       void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream);
 
 size_t bwd_workspace_bytes(const AttnShape& s);
 
 cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const void* o, const void* dout, const float* lse, void* dq,
+                       const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
+                       const float* lse, void* dq,
                        void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream);
 
 }  // namespace fa

@@ -42,10 +42,14 @@ def lib() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.fa_fwd.restype = i
+    L.fa_fwd_with_residual.argtypes = [vp] * 6 + [i, i, i, i, i, i, f, vp]
+    L.fa_fwd_with_residual.restype = i
     L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
     L.fa_bwd_workspace_bytes.restype = sz
     L.fa_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd.restype = i
+    L.fa_bwd_with_residual.argtypes = [vp] * 10 + [i, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_bwd_with_residual.restype = i
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_check_device_error.argtypes = [vp]
@@ -54,6 +58,8 @@ def lib() -> ctypes.CDLL:
     L.fa_set_watchdog_ns.restype = None
     L.fa_test_set_fault.argtypes = [i]
     L.fa_test_set_fault.restype = None
+    L.fa_profile_set_bwd_events.argtypes = [vp, vp]
+    L.fa_profile_set_bwd_events.restype = None
     _lib = L
     return L
 
@@ -89,24 +95,36 @@ def _shapes(q, k):
     return B, Hq, k.shape[1], N, d
 
 
-def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None) -> None:
-    """Forward pass into caller-owned ``o`` [B,Hq,N,d] bf16 and ``lse`` [B,Hq,N] fp32."""
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None, o_resid=None) -> None:
+    """Forward pass into caller-owned ``o`` [B,Hq,N,d] bf16 and ``lse`` [B,Hq,N] fp32.
+
+    With ``o_resid`` (bf16, like ``o``) this calls ``fa_fwd_with_residual``.
+    """
     B, Hq, Hkv, N, d = _shapes(q, k)
     bf = torch.bfloat16
-    args = [_check_tensor("q", q, bf, (B, Hq, N, d)), _check_tensor("k", k, bf, (B, Hkv, N, d)),
-            _check_tensor("v", v, bf, (B, Hkv, N, d)), _check_tensor("o", o, bf, (B, Hq, N, d)),
-            _check_tensor("lse", lse, torch.float32, (B, Hq, N))]
-    rc = lib().fa_fwd(*args, B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    qa, ka, va, oa = (_check_tensor("q", q, bf, (B, Hq, N, d)), _check_tensor("k", k, bf, (B, Hkv, N, d)),
+                      _check_tensor("v", v, bf, (B, Hkv, N, d)), _check_tensor("o", o, bf, (B, Hq, N, d)))
+    la = _check_tensor("lse", lse, torch.float32, (B, Hq, N))
+    tail = (B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if o_resid is None:
+        rc, name = lib().fa_fwd(qa, ka, va, oa, la, *tail), "fa_fwd"
+    else:
+        ra = _check_tensor("o_resid", o_resid, bf, (B, Hq, N, d))
+        rc, name = lib().fa_fwd_with_residual(qa, ka, va, oa, ra, la, *tail), "fa_fwd_with_residual"
     if rc != FA_OK:
-        raise FaError(rc, "fa_fwd")
+        raise FaError(rc, name)
 
 
 def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
     return int(lib().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
 
 
-def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None) -> None:
-    """Backward pass into caller-owned ``dq``, ``dk``, ``dv`` using ``workspace`` (uint8 CUDA tensor)."""
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None,
+           o_resid=None) -> None:
+    """Backward pass into caller-owned ``dq``, ``dk``, ``dv`` using ``workspace`` (uint8 CUDA tensor).
+
+    With ``o_resid`` (from :func:`fa_fwd`) this calls ``fa_bwd_with_residual``.
+    """
     B, Hq, Hkv, N, d = _shapes(q, k)
     bf = torch.bfloat16
     args = [_check_tensor("q", q, bf, (B, Hq, N, d)), _check_tensor("k", k, bf, (B, Hkv, N, d)),
@@ -118,10 +136,14 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, worksp
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
-    rc = lib().fa_bwd(*args, B, Hq, Hkv, N, d, int(bool(causal)), float(scale), workspace.data_ptr(),
-                      ws_bytes, _stream(stream))
+    tail = (B, Hq, Hkv, N, d, int(bool(causal)), float(scale), workspace.data_ptr(), ws_bytes, _stream(stream))
+    if o_resid is None:
+        rc, name = lib().fa_bwd(*args, *tail), "fa_bwd"
+    else:
+        ra = _check_tensor("o_resid", o_resid, bf, (B, Hq, N, d))
+        rc, name = lib().fa_bwd_with_residual(*args[:4], ra, *args[4:], *tail), "fa_bwd_with_residual"
     if rc != FA_OK:
-        raise FaError(rc, "fa_bwd")
+        raise FaError(rc, name)
 
 
 def fa_check_device_error(stream=None) -> int:
@@ -136,20 +158,30 @@ def fa_test_set_fault(code: int) -> None:
     lib().fa_test_set_fault(int(code))
 
 
+def fa_profile_set_bwd_events(after_pre=None, after_main=None) -> None:
+    """Hands two torch.cuda.Event objects (or None) to the timing hook."""
+    ptr = lambda e: None if e is None else e.cuda_event
+    lib().fa_profile_set_bwd_events(ptr(after_pre), ptr(after_main))
+
+
 # ------------------------------------------------------------ conveniences
 
-def attention_forward(q, k, v, causal: bool, scale: float | None = None, stream=None):
-    """Allocates ``o`` and ``lse`` with torch and runs :func:`fa_fwd`."""
+def attention_forward(q, k, v, causal: bool, scale: float | None = None, stream=None, residual: bool = False):
+    """Allocates ``o`` and ``lse`` with torch and runs :func:`fa_fwd`.
+
+    Returns ``(o, lse)``, or ``(o, lse, o_resid)`` when ``residual`` is true.
+    """
     B, Hq, Hkv, N, d = _shapes(q, k)
     scale = d ** -0.5 if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
-    fa_fwd(q, k, v, o, lse, causal, scale, stream)
-    return o, lse
+    o_resid = torch.empty_like(q) if residual else None
+    fa_fwd(q, k, v, o, lse, causal, scale, stream, o_resid=o_resid)
+    return (o, lse, o_resid) if residual else (o, lse)
 
 
 def attention_backward(q, k, v, o, dout, lse, causal: bool, scale: float | None = None, workspace=None,
-                       stream=None):
+                       stream=None, o_resid=None):
     """Allocates ``dq``, ``dk``, ``dv`` (and the workspace if not given) and runs :func:`fa_bwd`."""
     B, Hq, Hkv, N, d = _shapes(q, k)
     scale = d ** -0.5 if scale is None else scale
@@ -158,5 +190,5 @@ def attention_backward(q, k, v, o, dout, lse, causal: bool, scale: float | None 
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace, stream)
+    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace, stream, o_resid=o_resid)
     return dq, dk, dv

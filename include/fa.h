@@ -72,6 +72,18 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            int d, int causal, float scale, void* stream);
 
 /*
+ * Forward pass that also writes the bf16 rounding residual of o:
+ * o_resid = bf16(O - o), where O is the fp32 result before rounding and o is
+ * what fa_fwd writes. o + o_resid carries O to ~16 significant bits.
+ * fa_bwd_with_residual uses it to form D_i = sum_c dO_ic O_ic: D multiplies
+ * every error of O by dO and sums it over d, so the bf16 rounding of o alone
+ * shifts dQ and dK by ~1e-2 on peaky rows. Arguments as fa_fwd, plus
+ *   o_resid [B][Hq][N][d] (bf16, written; must not be NULL)
+ */
+int fa_fwd_with_residual(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse,
+                         int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for this shape: an fp32 row sum
  * D_i = sum_c dout_ic o_ic per query row, and an fp32 dQ accumulator
  * [B][Hq][N][d]. Returns 0 for an invalid or unsupported shape.
@@ -79,7 +91,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
 /*
- * Backward pass: gradients of sum(dout * o) with respect to q, k and v,
+ * Backward pass: gradients of sum(dout * O) with respect to q, k and v,
  * rebuilding P from q, k and lse tile by tile. Source: "FlashAttention:
  * IO-aware exact attention", "Four ideas" list, item "Recomputation in the
  * backward pass" (only the per-row logsumexp is kept from the forward pass
@@ -87,7 +99,9 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * definition above: dV = P^T dO, dP = dO V^T, D_i = sum_j P_ij dP_ij,
  * dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q, with the query
  * heads of a KV group summed into its dK, dV.
- *   q, k, v, o, dout, lse: as produced for / by fa_fwd (read only)
+ *   q, k, v, o, dout, lse: as produced for / by fa_fwd (read only). D_i is
+ *   formed from the bf16 o; see fa_bwd_with_residual for the variant that
+ *   removes o's rounding from D.
  *   dq [B][Hq][N][d], dk, dv [B][Hkv][N][d] (bf16, written)
  *   workspace: device memory of at least fa_bwd_workspace_bytes(...) bytes,
  *   16-byte aligned, owned by the caller, contents need not be initialised
@@ -96,6 +110,17 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
            void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass as fa_bwd, with D_i formed from o + o_resid (o_resid as
+ * written by fa_fwd_with_residual, read only, must not be NULL). This is the
+ * path whose gradients stay within 2e-2 (plus bf16 output rounding) of the
+ * exact gradients on peaky softmax rows.
+ */
+int fa_bwd_with_residual(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                         int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                         void* stream);
 
 /* Static text for a status code (for FA_ERR_CUDA: the last CUDA error seen by
  * this thread). Never NULL. */

@@ -48,8 +48,15 @@ def gpu_inputs(B, Hq, Hkv, N, d, seed, qk_gain=1.0, with_dout=True):
     return dev, ref
 
 
-def run_fwd(dev, causal, scale):
-    o, lse = fa.attention_forward(dev["q"], dev["k"], dev["v"], causal, scale)
+def run_fwd(dev, causal, scale, residual=False):
+    out = fa.attention_forward(dev["q"], dev["k"], dev["v"], causal, scale, residual=residual)
     torch.cuda.synchronize()
     assert fa.fa_check_device_error() == fa.FA_OK
-    return o, lse
+    return out
+
+
+def run_bwd(dev, o, lse, causal, scale, o_resid=None):
+    g = fa.attention_backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, causal, scale, o_resid=o_resid)
+    torch.cuda.synchronize()
+    assert fa.fa_check_device_error() == fa.FA_OK
+    return g

@@ -1,0 +1,79 @@
+"""Host-side logic of bench.py on the CPU: the max-over-ranks timing
+reduction with two gloo ranks, and the reference (oracle) arm's JSON line."""
+
+import json
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from exact_io_aware_56_b200 import WORKLOADS, Workload  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    r, w = bench.init_dist("gloo")
+    bench.barrier()
+    got = bench.max_over_ranks(10.0 * (r + 1))
+    bench.barrier()
+    import torch.distributed as dist
+
+    dist.destroy_process_group()
+    q.put((r, w, got))
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, 2, 20.0), (1, 2, 20.0)]
+
+
+def test_max_over_ranks_single_process_is_identity():
+    assert bench.max_over_ranks(3.5) == 3.5
+
+
+def test_reference_arm_json(monkeypatch, capsys):
+    tiny = Workload("tiny_ref", 1, 2, 1, 64, 64, True, True, seed=3)
+    monkeypatch.setitem(WORKLOADS, "tiny_ref", tiny)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--impl", "reference", "--workload", "tiny_ref", "--steps", "2", "--warmup", "1"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["config"]["workload"] == "tiny_ref"
+
+
+def test_reference_arm_other_ranks_exit_quietly(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_workload_flops():
+    w = WORKLOADS["fwdbwd_b2_h16_n8192_d128_causal_peaky"]
+    assert w.fwd_flops() == pytest.approx(549.755813888e9)
+    assert w.bwd_flops() == pytest.approx(2.5 * 549.755813888e9)
+    assert WORKLOADS["fwd_b1_h1_n128_d64"].fwd_flops() == 4 * 128 * 128 * 64
