@@ -122,6 +122,38 @@ int fa_bwd_with_residual(const void* q, const void* k, const void* v, const void
                          int N, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/*
+ * Size of the device array that fa_bwd_noalloc uses as its workspace.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * Backward pass as fa_bwd, without a workspace argument and without
+ * allocating anything. The source pages have no counterpart to this entry
+ * point; it exists for callers that cannot allocate device memory: hosts
+ * that hand a library only its input and output buffers (a fixed plugin
+ * signature with no workspace argument), or runtimes that budget all device
+ * memory themselves and forbid cudaMalloc, which also synchronises the
+ * device.
+ *   Arguments: as fa_bwd, minus workspace and workspace_bytes.
+ *   Scratch: a file-scope device array of FA_BWD_NOALLOC_SCRATCH_BYTES
+ *   (32 MiB) inside libfa, held by every GPU that loads it until the
+ *   process exits. The shape must satisfy
+ *   fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) <= FA_BWD_NOALLOC_SCRATCH_BYTES
+ *   (about 4 bytes * B*Hq*N*(d+1)); larger shapes return FA_ERR_UNSUPPORTED
+ *   before anything is launched.
+ *   The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture. No call allocates or frees memory.
+ *   Every call shares the array and it keeps the last call's contents; the
+ *   kernels rewrite what they read before using it. Calls whose kernels
+ *   overlap on the GPU (from several streams or host threads) race on the
+ *   array and give wrong results: serialise them.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                   void* stream);
+
 /* Static text for a status code (for FA_ERR_CUDA: the last CUDA error seen by
  * this thread). Never NULL. */
 const char* fa_status_string(int status);
