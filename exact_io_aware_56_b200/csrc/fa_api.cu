@@ -95,7 +95,9 @@ LaunchCtl make_ctl(const DevState* st) {
 
 }  // namespace
 
-bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows) {
+namespace {
+bool encode_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, int cols, int rows,
+                int outer, int box_cols, int box_rows) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -106,13 +108,25 @@ bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int
   if (!g_encode) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(outer)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, static_cast<cuuint64_t>(cols) * 2 * rows};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * elem_bytes,
+                           static_cast<cuuint64_t>(cols) * elem_bytes * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = g_encode(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, cols, rows, outer, 64, box_rows);
+}
+
+bool encode_f32_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_cols,
+                         int box_rows) {
+  if (box_cols * 4 > 128) return false;
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, cols, rows, outer, box_cols, box_rows);
 }
 
 }  // namespace fa

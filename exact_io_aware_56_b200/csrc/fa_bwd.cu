@@ -26,20 +26,29 @@
 //               dV_j += P^T dO_i          (P^T read from tensor memory)
 //               dK_j += dS^T Q_i          (dS^T from shared memory)
 //               dQ_i  = dS K_j            (same dS^T bytes read MN-major)
-//             and dQ_i is added to the fp32 accumulator with vector
-//             reductions. dK_j (times scale) and dV_j are written once.
+//             and dQ_i is added to the fp32 accumulator by TMA bulk
+//             reductions (cp.reduce.async.bulk.tensor ... add) of 128 x 32
+//             fp32 tiles staged in the dS^T buffer, which is free between
+//             the dQ MMA and the next tile's dP^T. dK_j (times scale) and
+//             dV_j are written once.
 //   bwd_post  dq = bf16(scale * accumulator).
 //
-// Warp roles of bwd_main (384 threads):
-//   warps 0-3   softmax-gradient warpgroup: thread = key row; writes P^T to
-//               tensor memory and dS^T to shared memory; epilogue stores dV.
-//   warps 4-7   dQ warpgroup: thread = query row; reads dQ_i out of tensor
-//               memory and reduces it into the accumulator; epilogue stores dK.
+// Warp roles of bwd_main (512 threads):
+//   warps 0-7   softmax-gradient warpgroups: thread = key row; warpgroup h
+//               handles query columns [64h, 64h+64) of each tile, writes its
+//               P^T to tensor memory and its dS^T half to shared memory;
+//               epilogue stores dV (half the columns each).
 //   warp 8      producer: K_j, V_j once; Q_i, dO_i by TMA and L_i, D_i by
 //               plain loads into a two-stage ring.
-//   warp 9      tensor-memory owner and MMA issuer.
-// Tensor memory: [0,128) S^T | [128,256) dP^T, then P^T (bf16) in its first
-// 64 columns, then dQ_i | dV_j (D columns) | dK_j (D columns).
+//   warp 9      tensor-memory owner and MMA issuer. dV and dK of a query
+//               half are issued as soon as that half's P^T and dS^T exist.
+//   warps 10-11 idle (keep the third warpgroup whole).
+//   warps 12-15 dQ warpgroup: thread = query row; reads dQ_i out of tensor
+//               memory, stages it in shared memory and issues the bulk
+//               reductions into the accumulator; epilogue stores dK.
+// Tensor memory: [0,128) S^T | [128,256) dP^T, then P^T (bf16: query half h
+// in columns [64h, 64h+32) of the block), then dQ_i | dV_j (D columns) |
+// dK_j (D columns).
 // Every tcgen05 operation of the MMA thread completes in issue order, which
 // orders P^T reads before the dQ write into the same columns.
 
@@ -53,7 +62,8 @@ namespace fa {
 namespace {
 
 constexpr int kB = 128;  // rows per Q tile and per K/V tile
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kDqWarp0 = 12;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -92,7 +102,7 @@ struct BwdArgs {
 struct BwdBars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, dp_full, p_ready, ds_free, dq_full, dq_empty, acc_final, drain;
+  uint64_t s_full, dp_full, p_ready[2], ds_free, dq_full, dq_empty, acc_final, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -107,11 +117,39 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// out[tile at (c0, c1, c2)] += smem tile, fp32 add, as one bulk operation.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(m),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void dq_group_sync() {  // the 128 threads of the dQ warpgroup
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// AND of `v` over the 128 threads of the dQ warpgroup (also a barrier), so
+// that the four warps always take the same branch around dq_group_sync.
+__device__ __forceinline__ bool dq_group_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const BwdArgs a) {
+                    const __grid_constant__ CUtensorMap tmDQacc, const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -129,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // Work unit: (batch, KV head, key tile j); the longest units (smallest j
-  // when causal) get the lowest block indices.
+  // when causal) get the lowest block indices (longest-processing-time order).
   const int bkv = blockIdx.x % a.BHkv;
   const int j = blockIdx.x / a.BHkv;
   const int r = a.Hq / a.Hkv;
@@ -147,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_ready, kB);
+    mbar_init(&bars->p_ready[0], kB);
+    mbar_init(&bars->p_ready[1], kB);
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, kB);
@@ -264,13 +303,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int it = 0; ok && it < n_it; ++it) {
         const int s = it & 1;
-        if (!(ok = wait_bar(&bars->p_ready, it & 1, w))) break;
-        tc_fence_after();
         const uint32_t q = sQ + s * C::kTileBytes, o = sDO + s * C::kTileBytes;
+        // dV += P^T dO and dK += dS^T Q, query half by query half (K = 64 each).
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!(ok = wait_bar(&bars->p_ready[hf], it & 1, w))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < kB / 16; ++k) mma_ts(tDV, tDP + k * 8, mdesc(o, k), id_dv, (it > 0 || k > 0));
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = 4 * hf + kk;
+            mma_ts(tDV, tDP + 64 * hf + 8 * kk, mdesc(o, k), id_dv, (it > 0 || k > 0));
+          }
 #pragma unroll
-        for (int k = 0; k < kB / 16; ++k) mma_ss(tDK, kdesc(sDS, k), mdesc(q, k), id_dk, (it > 0 || k > 0));
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = 4 * hf + kk;
+            mma_ss(tDK, kdesc(sDS, k), mdesc(q, k), id_dk, (it > 0 || k > 0));
+          }
+        }
+        if (!ok) break;
 #pragma unroll
         for (int k = 0; k < kB / 16; ++k) mma_ss(tDP, mdesc(sDS, k), mdesc(sK, k), id_dq, k > 0);
         mma_commit(&bars->dq_full);
@@ -290,75 +339,89 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bars->drain);
       drain_bar(&bars->drain, 0, w);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------- P^T and dS^T (key rows)
+    const int hf = warp >> 2;                              // query half of this warpgroup
     const int quad = warp & 3;
     const int kr = quad * 32 + lane;                       // key row in tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS;
-    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const uint32_t tS = tmem + lane_off + C::kColS + 64 * hf;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * hf;
     const float sl2 = a.scale_log2;
-    uint8_t* ds_row = smem + C::kOffDS + kr * 128;         // row kr of both 64-column boxes
+    uint8_t* ds_row = smem + C::kOffDS + hf * (kB * 128) + kr * 128;  // row kr of box hf
     const uint32_t sw = static_cast<uint32_t>(kr & 7);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int s = it & 1;
       const int i = i0 + it % nqi;
-      const float* l2 = sLD + s * 2 * kB;
+      const float* l2 = sLD + s * 2 * kB + 64 * hf;
       const float* dd = l2 + kB;
       // q_full orders the producer's plain stores of L and D before these reads.
+      // (dp_full also orders this tile's dS^T writes after the dQ warpgroup's
+      // use of the same buffer as staging for the previous tile.)
       ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[s], (it >> 1) & 1, w));
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full, it & 1, w));
       if (ok && it > 0) ok = __all_sync(0xffffffffu, wait_bar(&bars->ds_free, (it - 1) & 1, w));
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->dp_full, it & 1, w));
       if (!ok) break;
       tc_fence_after();
-      const bool diag = CAUSAL && (i == j);
+      const int diag_lim = (CAUSAL && i == j) ? kr - 64 * hf : -1;  // local queries < diag_lim are masked
 #pragma unroll
-      for (int c = 0; c < kB / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + c * 32, sv);
         tmem_ld32(tDP + c * 32, dv);
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int q0 = c * 32 + 2 * e;
-          float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l2[q0]));
-          float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l2[q0 + 1]));
-          if (diag) {
-            if (q0 < kr) p0 = 0.f;
-            if (q0 + 1 < kr) p1 = 0.f;
+        for (int x = 0; x < 8; ++x) {
+          const int q0 = c * 32 + 4 * x;                   // local query of this group of 4
+          const float4 lq = *reinterpret_cast<const float4*>(l2 + q0);
+          const float4 dq = *reinterpret_cast<const float4*>(dd + q0);
+          float p[4] = {ex2(fmaf(__uint_as_float(sv[4 * x]), sl2, -lq.x)),
+                        ex2(fmaf(__uint_as_float(sv[4 * x + 1]), sl2, -lq.y)),
+                        ex2(fmaf(__uint_as_float(sv[4 * x + 2]), sl2, -lq.z)),
+                        ex2(fmaf(__uint_as_float(sv[4 * x + 3]), sl2, -lq.w))};
+          if (q0 + 3 < diag_lim) {
+            p[0] = p[1] = p[2] = p[3] = 0.f;
+          } else if (q0 < diag_lim) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (q0 + e < diag_lim) p[e] = 0.f;
           }
-          const float d0 = p0 * (__uint_as_float(dv[2 * e]) - dd[q0]);
-          const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - dd[q0 + 1]);
-          pk[e] = pack_bf16x2(p0, p1);
-          dk[e] = pack_bf16x2(d0, d1);
+          const float g0 = p[0] * (__uint_as_float(dv[4 * x]) - dq.x);
+          const float g1 = p[1] * (__uint_as_float(dv[4 * x + 1]) - dq.y);
+          const float g2 = p[2] * (__uint_as_float(dv[4 * x + 2]) - dq.z);
+          const float g3 = p[3] * (__uint_as_float(dv[4 * x + 3]) - dq.w);
+          pk[2 * x] = pack_bf16x2(p[0], p[1]);
+          pk[2 * x + 1] = pack_bf16x2(p[2], p[3]);
+          dk[2 * x] = pack_bf16x2(g0, g1);
+          dk[2 * x + 1] = pack_bf16x2(g2, g3);
         }
-        // P^T chunk -> tensor memory columns [16c, 16c+16) of the dP^T block
-        // (those columns' dP^T values were consumed by this or an earlier chunk).
+        // P^T chunk -> columns [16c, 16c+16) of this half's dP^T columns
+        // (their dP^T values were loaded by this or the previous chunk).
         tmem_st16(tDP + c * 16, pk);
-        // dS^T chunk: queries [32c, 32c+32) of key row kr, 128-byte swizzled.
-        uint8_t* box = ds_row + (c >> 1) * (kB * 128);
+        // dS^T chunk: local queries [32c, 32c+32) of key row kr, 128-byte swizzled.
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t chunk = static_cast<uint32_t>((c & 1) * 4 + u);
+          const uint32_t chunk = static_cast<uint32_t>(c * 4 + u);
           uint4 val = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-          *reinterpret_cast<uint4*>(box + ((chunk ^ sw) << 4)) = val;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ sw) << 4)) = val;
         }
       }
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready);
+      mbar_arrive(&bars->p_ready[hf]);
     }
-    // Epilogue: dV_j rows (this thread's key row).
+    // Epilogue: dV_j rows (this thread's key row), half of the columns per warpgroup.
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
       tc_fence_after();
       const int key = j * kB + kr;
       __nv_bfloat16* dst = a.dv + (static_cast<size_t>(bkv) * a.N + key) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c = hf * (D / 64) + cc;
         uint32_t vv[32];
         tmem_ld32(tmem + lane_off + C::kColDV + c * 32, vv);
         uint4 o4[4];
@@ -371,35 +434,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp >= kDqWarp0) {
     // ----------------------------------------------- dQ_i readout (query rows)
     const int quad = warp & 3;
     const int qr = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tDQ = tmem + lane_off + C::kColDP;
+    uint8_t* stage = smem + C::kOffDS;                     // two 128 x 32 fp32 boxes, 128-byte swizzled
+    const uint32_t sw = static_cast<uint32_t>(qr & 7);
+    const bool leader = (warp == kDqWarp0 && lane == 0);
+    if (leader) tma_prefetch_desc(&tmDQacc);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      ok = __all_sync(0xffffffffu, wait_bar(&bars->dq_full, it & 1, w));
+      ok = dq_group_all(wait_bar(&bars->dq_full, it & 1, w));
       if (!ok) break;
       tc_fence_after();
       const int h = g * r + it / nqi;
       const int i = i0 + it % nqi;
-      const int row = i * kB + qr;
-      float* dst = a.dq_acc + ((static_cast<size_t>(b) * a.Hq + h) * a.N + row) * D;
+      const int bh = b * a.Hq + h;
+      // The dQ and dK MMAs that read dS^T have completed (dq_full), and the
+      // softmax-gradient warps write dS^T again only after the next dP^T,
+      // which waits for dq_empty: the buffer is this warpgroup's until then.
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t vv[32];
-        tmem_ld32(tDQ + c * 32, vv);
-        if (row < a.N) {
+      for (int rd = 0; rd < D / 64; ++rd) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            red_add_v4(dst + c * 32 + 4 * e, __uint_as_float(vv[4 * e]), __uint_as_float(vv[4 * e + 1]),
-                       __uint_as_float(vv[4 * e + 2]), __uint_as_float(vv[4 * e + 3]));
+        for (int bx = 0; bx < 2; ++bx) {
+          uint32_t vv[32];
+          tmem_ld32(tDQ + rd * 64 + bx * 32, vv);
+          uint8_t* row = stage + bx * (kB * 128) + qr * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(u) ^ sw) << 4)) =
+                make_uint4(vv[4 * u], vv[4 * u + 1], vv[4 * u + 2], vv[4 * u + 3]);
         }
+        fence_async_smem();
+        dq_group_sync();
+        if (leader) {
+          // Rows past N fall outside the tensor map's row extent and are dropped.
+          tma_reduce_add_3d(&tmDQacc, stage, rd * 64, i * kB, bh);
+          tma_reduce_add_3d(&tmDQacc, stage + kB * 128, rd * 64 + 32, i * kB, bh);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        dq_group_sync();
       }
       tc_fence_before();
       mbar_arrive(&bars->dq_empty);
     }
+    if (leader) bulk_wait0();
     // Epilogue: dK_j = scale * accumulated dS^T Q (this thread's key row).
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
@@ -498,10 +580,12 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
                          const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
                          cudaStream_t stream) {
   using C = BwdCfg<D>;
+  CUtensorMap tdq;
   const long long rows = static_cast<long long>(s.B) * s.Hq * s.N;
   float* dsum = static_cast<float*>(workspace);
   const size_t dsum_bytes = ((static_cast<size_t>(rows) * 4 + 255) / 256) * 256;
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsum_bytes);
+  if (!encode_f32_tile_map(&tdq, dq_acc, s.d, s.N, s.B * s.Hq, 32, kB)) return cudaErrorInvalidValue;
 
   bwd_pre_kernel<D><<<grid_for(rows, 8, 148 * 64), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_resid),
@@ -530,7 +614,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.nk) * a.BHkv;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ctl.ev_after_main && (e = cudaEventRecord(ctl.ev_after_main, stream)) != cudaSuccess) return e;

@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Work unit: (batch*head, pair of Q tiles). The heaviest pairs (largest
   // query index, most K/V tiles when causal) get the lowest block indices so
-  // they start first; heads sharing a KV head are adjacent.
+  // they start first (longest-processing-time order); heads sharing a KV
+  // head are adjacent.
   const int bh = blockIdx.x % a.BH;
   const int pair = a.n_pairs - 1 - blockIdx.x / a.BH;
   const int h = bh % a.Hq;

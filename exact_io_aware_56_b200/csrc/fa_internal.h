@@ -27,6 +27,10 @@ struct LaunchCtl {
 // 64 columns x box_rows rows and 128-byte swizzle. Returns false on failure.
 bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows);
 
+// Same for an fp32 tensor, box of box_cols x box_rows (box_cols * 4 <= 128).
+bool encode_f32_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_cols,
+                         int box_rows);
+
 // o_resid may be null (no residual written).
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream);
