@@ -17,40 +17,38 @@
 //             bf16 rounding of O alone moves D by ~1e-2 at d = 128.
 //   bwd_main  one CTA per (batch, KV head, 128-key tile j). K_j and V_j stay in
 //             shared memory; the CTA loops over the query heads of the KV
-//             group and the 128-row query tiles i that can see tile j
-//             (i >= j when causal). Per (head, i):
-//               S^T  = K_j Q_i^T          (tcgen05 -> tensor memory)
+//             group and the 64-row query tiles i that can see tile j
+//             (i >= 2j when causal). Per (head, i):
+//               S^T  = K_j Q_i^T          (tcgen05 -> tensor memory, M=128 N=64)
 //               dP^T = V_j dO_i^T         (tcgen05 -> tensor memory)
 //               P^T  = 2^(S^T scale log2e - L_i log2e), dS^T = P^T o (dP^T - D_i)
 //                                         (one thread per key row)
 //               dV_j += P^T dO_i          (P^T read from tensor memory)
 //               dK_j += dS^T Q_i          (dS^T from shared memory)
-//               dQ_i  = dS K_j            (same dS^T bytes read MN-major)
-//             and dQ_i is added to the fp32 accumulator by TMA bulk
-//             reductions (cp.reduce.async.bulk.tensor ... add) of 128 x 32
-//             fp32 tiles staged in the dS^T buffer, which is free between
-//             the dQ MMA and the next tile's dP^T. dK_j (times scale) and
-//             dV_j are written once.
+//               dQ_i^T = K_j^T dS_i^T     (M = d: one thread per column of dQ)
+//             dQ_i is staged in shared memory and added to the fp32
+//             accumulator by TMA bulk reductions, which overlap the next
+//             tiles. dK_j (times scale) and dV_j are written once.
 //   bwd_post  dq = bf16(scale * accumulator).
 //
 // Warp roles of bwd_main (512 threads):
-//   warps 0-7   softmax-gradient warpgroups: thread = key row; warpgroup h
-//               handles query columns [64h, 64h+64) of each tile, writes its
-//               P^T to tensor memory and its dS^T half to shared memory;
-//               epilogue stores dV (half the columns each).
+//   warps 0-3   softmax-gradient warpgroup for even query tiles (buffer 0),
+//   warps 4-7   the same for odd tiles (buffer 1): thread = key row; writes
+//               P^T to tensor memory and dS^T to shared memory; epilogue
+//               stores dV (half of the columns each).
 //   warp 8      producer: K_j, V_j once; Q_i, dO_i by TMA and L_i, D_i by
-//               plain loads into a two-stage ring.
-//   warp 9      tensor-memory owner and MMA issuer. dV and dK of a query
-//               half are issued as soon as that half's P^T and dS^T exist.
+//               plain loads into a three-stage ring.
+//   warp 9      tensor-memory owner and MMA issuer.
 //   warps 10-11 idle (keep the third warpgroup whole).
-//   warps 12-15 dQ warpgroup: thread = query row; reads dQ_i out of tensor
-//               memory, stages it in shared memory and issues the bulk
-//               reductions into the accumulator; epilogue stores dK.
-// Tensor memory: [0,128) S^T | [128,256) dP^T, then P^T (bf16: query half h
-// in columns [64h, 64h+32) of the block), then dQ_i | dV_j (D columns) |
-// dK_j (D columns).
-// Every tcgen05 operation of the MMA thread completes in issue order, which
-// orders P^T reads before the dQ write into the same columns.
+//   warps 12-15 dQ warpgroup: thread = column c of dQ; reads dQ_i^T out of
+//               tensor memory, stages it and issues the bulk reductions;
+//               epilogue stores dK.
+// Tensor memory (512 columns): S^T[2] (64 each) | dP^T[2] (64 each; P^T in
+// bf16 over its first 32 columns, then dQ_i^T over all 64) | dV (D) | dK (D).
+// S^T and dP^T are double-buffered so that one warpgroup's softmax-gradient
+// work overlaps the MMAs of the other's tile. Every tcgen05 operation of the
+// MMA thread completes in issue order, which orders the P^T reads of dV
+// before the dQ^T write into the same columns.
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -61,25 +59,32 @@
 namespace fa {
 namespace {
 
-constexpr int kB = 128;  // rows per Q tile and per K/V tile
+constexpr int kKT = 128;   // keys per key tile (MMA M of the key-side products)
+constexpr int kQT = 64;    // queries per query tile
 constexpr int kThreads = 512;
-constexpr int kDqWarp0 = 12;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kDqWarp0 = 12;
+constexpr int kQStages = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kBoxBytes = kB * 64 * 2;
-  static constexpr int kTileBytes = kBoxBytes * (D / 64);  // one 128 x D bf16 tile
-  static constexpr int kStages = 2;
+  static constexpr int kKBox = kKT * 128;                  // one 64-column box of a 128-row tile
+  static constexpr int kKTile = kKBox * (D / 64);          // K_j or V_j
+  static constexpr int kQBox = kQT * 128;                  // one 64-column box of a 64-row tile
+  static constexpr int kQTile = kQBox * (D / 64);          // Q_i or dO_i
+  static constexpr int kDSTile = kKT * kQT * 2;            // dS^T: 128 keys x 64 queries bf16 (one box)
+  static constexpr int kStBox = kQT * 128;                 // staging: 64 rows x 32 fp32
+  static constexpr int kStTile = kStBox * (D / 32);        // dQ_i fp32, 64 x D
   static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kTileBytes;
-  static constexpr int kOffQ = kOffV + kTileBytes;                  // [stage] Q_i
-  static constexpr int kOffDO = kOffQ + kStages * kTileBytes;       // [stage] dO_i
-  static constexpr int kOffDS = kOffDO + kStages * kTileBytes;      // dS^T, 128 x 128 bf16
-  static constexpr int kOffLD = kOffDS + 2 * kBoxBytes;             // [stage] L2[128], D[128]
-  static constexpr int kOffBar = kOffLD + kStages * 2 * kB * 4;
+  static constexpr int kOffV = kOffK + kKTile;
+  static constexpr int kOffQ = kOffV + kKTile;
+  static constexpr int kOffDO = kOffQ + kQStages * kQTile;
+  static constexpr int kOffDS = kOffDO + kQStages * kQTile;
+  static constexpr int kOffST = kOffDS + 2 * kDSTile;
+  static constexpr int kOffLD = kOffST + kStTile;          // [stage] L2[64], D[64]
+  static constexpr int kOffBar = kOffLD + kQStages * 2 * kQT * 4;
   static constexpr int kUsed = kOffBar + 256;
   static constexpr int kSmemBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
   static constexpr uint32_t kTmemCols = 512;
@@ -91,7 +96,6 @@ struct BwdCfg {
 struct BwdArgs {
   const float* lse;
   const float* dsum;    // D_i, fp32 [B*Hq*N]
-  float* dq_acc;        // fp32 [B*Hq*N*d]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Hq, Hkv, BHkv, nk, nq;
@@ -101,20 +105,15 @@ struct BwdArgs {
 
 struct BwdBars {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, dp_full, p_ready[2], ds_free, dq_full, dq_empty, acc_final, drain;
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t s_full[2], dp_full[2], p_ready[2], ds_free[2], dq_full[2], dq_empty[2];
+  uint64_t acc_final, drain;
   uint32_t tmem_base;
   int abort;
 };
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
 }
 
 // out[tile at (c0, c1, c2)] += smem tile, fp32 add, as one bulk operation.
@@ -173,23 +172,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = a.Hq / a.Hkv;
   const int b = bkv / a.Hkv;
   const int g = bkv % a.Hkv;
-  const int i0 = CAUSAL ? j : 0;
-  const int nqi = a.nq - i0;     // query tiles per head
-  const int n_it = r * nqi;      // (head, query tile) iterations
+  const int i0 = CAUSAL ? 2 * j : 0;   // first 64-row query tile that sees key tile j
+  const int nqi = a.nq - i0;           // query tiles per head
+  const int n_it = r * nqi;            // (head, query tile) iterations
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < kQStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_ready[0], kB);
-    mbar_init(&bars->p_ready[1], kB);
-    mbar_init(&bars->ds_free, 1);
-    mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_empty, kB);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->dp_full[x], 1);
+      mbar_init(&bars->p_ready[x], kKT);
+      mbar_init(&bars->ds_free[x], 1);
+      mbar_init(&bars->dq_full[x], 1);
+      mbar_init(&bars->dq_empty[x], 128);
+    }
     mbar_init(&bars->acc_final, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -213,7 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    int q_last[2] = {-1, -1};
+    int q_last[kQStages];
+#pragma unroll
+    for (int s = 0; s < kQStages; ++s) q_last[s] = -1;
     bool kv_issued = false;
     bool ok = true;
     if (lane == 0) {
@@ -221,31 +223,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kKTile);
       for (int x = 0; x < D / 64; ++x) {
-        tma_load_3d(&tmK, &bars->kv_full, smem + C::kOffK + x * C::kBoxBytes, x * 64, j * kB, bkv);
-        tma_load_3d(&tmV, &bars->kv_full, smem + C::kOffV + x * C::kBoxBytes, x * 64, j * kB, bkv);
+        tma_load_3d(&tmK, &bars->kv_full, smem + C::kOffK + x * C::kKBox, x * 64, j * kKT, bkv);
+        tma_load_3d(&tmV, &bars->kv_full, smem + C::kOffV + x * C::kKBox, x * 64, j * kKT, bkv);
       }
       kv_issued = true;
     }
     for (int it = 0; it < n_it; ++it) {
-      const int s = it & 1;
-      const int u = it >> 1;
-      if (it >= 2) {
+      const int s = it % kQStages;
+      const int u = it / kQStages;
+      if (it >= kQStages) {
         ok = __all_sync(0xffffffffu, wait_bar(&bars->q_empty[s], (u - 1) & 1, w));
         if (!ok) break;
       }
       const int h = g * r + it / nqi;
       const int i = i0 + it % nqi;
       const int bh = b * a.Hq + h;
-      // L (in log2 units) and D for the 128 query rows of this tile; rows
+      // L (in log2 units) and D for the 64 query rows of this tile; rows
       // past N get L = +inf so that their P is exactly 0.
-      float* l2 = sLD + s * 2 * kB;
-      float* dd = l2 + kB;
+      float* l2 = sLD + s * 2 * kQT;
+      float* dd = l2 + kQT;
 #pragma unroll
-      for (int e = 0; e < kB / 32; ++e) {
+      for (int e = 0; e < kQT / 32; ++e) {
         const int rr = e * 32 + lane;
-        const int row = i * kB + rr;
+        const int row = i * kQT + rr;
         const bool in = row < a.N;
         const size_t idx = static_cast<size_t>(bh) * a.N + row;
         l2[rr] = in ? a.lse[idx] * kLog2e : CUDART_INF_F;
@@ -253,86 +255,87 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::kTileBytes);
+        mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::kQTile);
         for (int x = 0; x < D / 64; ++x) {
-          tma_load_3d(&tmQ, &bars->q_full[s], smem + C::kOffQ + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                      i * kB, bh);
-          tma_load_3d(&tmDO, &bars->q_full[s], smem + C::kOffDO + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                      i * kB, bh);
+          tma_load_3d(&tmQ, &bars->q_full[s], smem + C::kOffQ + s * C::kQTile + x * C::kQBox, x * 64, i * kQT,
+                      bh);
+          tma_load_3d(&tmDO, &bars->q_full[s], smem + C::kOffDO + s * C::kQTile + x * C::kQBox, x * 64, i * kQT,
+                      bh);
         }
         q_last[s] = u;
       }
     }
     if (lane == 0) {
       if (kv_issued) drain_bar(&bars->kv_full, 0, w);
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < kQStages; ++s)
         if (q_last[s] >= 0) drain_bar(&bars->q_full[s], q_last[s] & 1, w);
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t id_sdp = idesc_bf16(kB, kB, false, false);  // S^T, dP^T
-      constexpr uint32_t id_dv = idesc_bf16(kB, D, false, true);     // dV (A in tensor memory)
-      constexpr uint32_t id_dk = idesc_bf16(kB, D, false, true);     // dK
-      constexpr uint32_t id_dq = idesc_bf16(kB, D, true, true);      // dQ (A = dS, MN-major)
-      const uint32_t tS = tmem + C::kColS, tDP = tmem + C::kColDP;
+      constexpr uint32_t id_sdp = idesc_bf16(kKT, kQT, false, false);  // S^T, dP^T: 128 x 64
+      constexpr uint32_t id_dvk = idesc_bf16(kKT, D, false, true);     // dV (A in TMEM), dK
+      constexpr uint32_t id_dq = idesc_bf16(128, kQT, true, true);     // dQ^T: A = K^T, B = dS^T
+      // K-major operand of a 128-row tile (64-column boxes kKBox apart).
+      auto kdesc_k = [](uint32_t base, int k) {
+        return sdesc_sw128(base + (k / 4) * (kKT * 128) + (k % 4) * 32, 16, 1024);
+      };
+      // K-major operand of a 64-row tile.
+      auto kdesc_q = [](uint32_t base, int k) {
+        return sdesc_sw128(base + (k / 4) * (kQT * 128) + (k % 4) * 32, 16, 1024);
+      };
+      // MN-major operands, K step k (16 rows): 64-column chunks `lbo` apart.
+      auto mdesc = [](uint32_t base, int k, uint32_t lbo) { return sdesc_sw128(base + k * 2048, lbo, 1024); };
+      auto issue_sdp = [&](int it) {
+        const int x = it & 1;
+        const uint32_t q = sQ + (it % kQStages) * C::kQTile, o = sDO + (it % kQStages) * C::kQTile;
+        const uint32_t tS = tmem + C::kColS + 64 * x, tDP = tmem + C::kColDP + 64 * x;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) mma_ss(tS, kdesc_k(sK, k), kdesc_q(q, k), id_sdp, k > 0);
+        mma_commit(&bars->s_full[x]);
+        return [=] {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc_k(sV, k), kdesc_q(o, k), id_sdp, k > 0);
+        };
+      };
       const uint32_t tDV = tmem + C::kColDV, tDK = tmem + C::kColDK;
-      auto kdesc = [](uint32_t base, int k) {  // K-major operand, K step k (16 elements)
-        return sdesc_sw128(base + (k / 4) * (kB * 128) + (k % 4) * 32, 16, 1024);
-      };
-      auto mdesc = [](uint32_t base, int k) {  // MN-major operand, K step k (16 rows)
-        return sdesc_sw128(base + k * 2048, kB * 128, 1024);
-      };
-      auto issue_sdp = [&](int s) {
-        const uint32_t q = sQ + s * C::kTileBytes;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tS, kdesc(sK, k), kdesc(q, k), id_sdp, k > 0);
-        mma_commit(&bars->s_full);
-      };
-      auto issue_dp = [&](int s) {
-        const uint32_t o = sDO + s * C::kTileBytes;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc(sV, k), kdesc(o, k), id_sdp, k > 0);
-        mma_commit(&bars->dp_full);
-      };
-      bool ok = wait_bar(&bars->kv_full, 0, w) && wait_bar(&bars->q_full[0], 0, w);
-      if (ok) {
+      bool ok = wait_bar(&bars->kv_full, 0, w);
+      for (int it = 0; ok && it < 2 && it < n_it; ++it) {
+        if (!(ok = wait_bar(&bars->q_full[it % kQStages], (it / kQStages) & 1, w))) break;
         tc_fence_after();
-        issue_sdp(0);
-        issue_dp(0);
+        auto dp = issue_sdp(it);
+        dp();
+        mma_commit(&bars->dp_full[it & 1]);
       }
       for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it & 1;
-        const uint32_t q = sQ + s * C::kTileBytes, o = sDO + s * C::kTileBytes;
-        // dV += P^T dO and dK += dS^T Q, query half by query half (K = 64 each).
-        for (int hf = 0; hf < 2; ++hf) {
-          if (!(ok = wait_bar(&bars->p_ready[hf], it & 1, w))) break;
-          tc_fence_after();
+        const int x = it & 1;
+        const int s = it % kQStages;
+        const uint32_t q = sQ + s * C::kQTile, o = sDO + s * C::kQTile;
+        const uint32_t tDP = tmem + C::kColDP + 64 * x;
+        const uint32_t ds = sDS + x * C::kDSTile;
+        if (!(ok = wait_bar(&bars->p_ready[x], (it >> 1) & 1, w))) break;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int k = 4 * hf + kk;
-            mma_ts(tDV, tDP + 64 * hf + 8 * kk, mdesc(o, k), id_dv, (it > 0 || k > 0));
-          }
+        for (int k = 0; k < kQT / 16; ++k)  // dV += P^T dO (K = 64 queries)
+          mma_ts(tDV, tDP + 8 * k, mdesc(o, k, C::kQBox), id_dvk, (it > 0 || k > 0));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int k = 4 * hf + kk;
-            mma_ss(tDK, kdesc(sDS, k), mdesc(q, k), id_dk, (it > 0 || k > 0));
-          }
-        }
-        if (!ok) break;
+        for (int k = 0; k < kQT / 16; ++k)  // dK += dS^T Q
+          mma_ss(tDK, kdesc_q(ds, k), mdesc(q, k, C::kQBox), id_dvk, (it > 0 || k > 0));
 #pragma unroll
-        for (int k = 0; k < kB / 16; ++k) mma_ss(tDP, mdesc(sDS, k), mdesc(sK, k), id_dq, k > 0);
-        mma_commit(&bars->dq_full);
-        mma_commit(&bars->ds_free);
+        for (int k = 0; k < kKT / 16; ++k)  // dQ^T = K^T dS^T (K = 128 keys)
+          mma_ss(tDP, mdesc(sK, k, C::kKBox), mdesc(ds, k, C::kKBox), id_dq, k > 0);
+        mma_commit(&bars->dq_full[x]);
+        mma_commit(&bars->ds_free[x]);
         mma_commit(&bars->q_empty[s]);
-        if (it + 1 < n_it) {
-          const int s1 = (it + 1) & 1;
-          if (!(ok = wait_bar(&bars->q_full[s1], ((it + 1) >> 1) & 1, w))) break;
+        const int nx = it + 2;
+        if (nx < n_it) {
+          if (!(ok = wait_bar(&bars->q_full[nx % kQStages], (nx / kQStages) & 1, w))) break;
           tc_fence_after();
-          issue_sdp(s1);
-          if (!(ok = wait_bar(&bars->dq_empty, it & 1, w))) break;
+          auto dp = issue_sdp(nx);
+          if (!(ok = wait_bar(&bars->dq_empty[x], (it >> 1) & 1, w))) break;
           tc_fence_after();
-          issue_dp(s1);
+          dp();
+          mma_commit(&bars->dp_full[x]);
         }
       }
       mma_commit(&bars->acc_final);
@@ -341,87 +344,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 8) {
     // ------------------------------------------- P^T and dS^T (key rows)
-    const int hf = warp >> 2;                              // query half of this warpgroup
+    const int x = warp >> 2;                               // buffer = parity of the tiles handled
     const int quad = warp & 3;
     const int kr = quad * 32 + lane;                       // key row in tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS + 64 * hf;
-    const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * hf;
+    const uint32_t tS = tmem + lane_off + C::kColS + 64 * x;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * x;
     const float sl2 = a.scale_log2;
-    uint8_t* ds_row = smem + C::kOffDS + hf * (kB * 128) + kr * 128;  // row kr of box hf
+    uint8_t* ds_row = smem + C::kOffDS + x * C::kDSTile + kr * 128;
     const uint32_t sw = static_cast<uint32_t>(kr & 7);
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it & 1;
+    for (int it = x; it < n_it; it += 2) {
+      const int s = it % kQStages;
       const int i = i0 + it % nqi;
-      const float* l2 = sLD + s * 2 * kB + 64 * hf;
-      const float* dd = l2 + kB;
+      const uint32_t par = (it >> 1) & 1;
+      const float* l2 = sLD + s * 2 * kQT;
+      const float* dd = l2 + kQT;
       // q_full orders the producer's plain stores of L and D before these reads.
-      // (dp_full also orders this tile's dS^T writes after the dQ warpgroup's
-      // use of the same buffer as staging for the previous tile.)
-      ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[s], (it >> 1) & 1, w));
-      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full, it & 1, w));
-      if (ok && it > 0) ok = __all_sync(0xffffffffu, wait_bar(&bars->ds_free, (it - 1) & 1, w));
-      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->dp_full, it & 1, w));
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[s], (it / kQStages) & 1, w));
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[x], par, w));
+      if (ok && it >= 2) ok = __all_sync(0xffffffffu, wait_bar(&bars->ds_free[x], par ^ 1, w));
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->dp_full[x], par, w));
       if (!ok) break;
       tc_fence_after();
-      const int diag_lim = (CAUSAL && i == j) ? kr - 64 * hf : -1;  // local queries < diag_lim are masked
+      // Local query ql is masked when its position is below this key's.
+      const int diag_lim = CAUSAL ? kKT * j + kr - kQT * i : -1;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kQT / 32; ++c) {
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + c * 32, sv);
         tmem_ld32(tDP + c * 32, dv);
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int q0 = c * 32 + 4 * x;                   // local query of this group of 4
+        for (int y = 0; y < 8; ++y) {
+          const int q0 = c * 32 + 4 * y;
           const float4 lq = *reinterpret_cast<const float4*>(l2 + q0);
           const float4 dq = *reinterpret_cast<const float4*>(dd + q0);
-          float p[4] = {ex2(fmaf(__uint_as_float(sv[4 * x]), sl2, -lq.x)),
-                        ex2(fmaf(__uint_as_float(sv[4 * x + 1]), sl2, -lq.y)),
-                        ex2(fmaf(__uint_as_float(sv[4 * x + 2]), sl2, -lq.z)),
-                        ex2(fmaf(__uint_as_float(sv[4 * x + 3]), sl2, -lq.w))};
-          if (q0 + 3 < diag_lim) {
-            p[0] = p[1] = p[2] = p[3] = 0.f;
-          } else if (q0 < diag_lim) {
+          float p[4] = {ex2(fmaf(__uint_as_float(sv[4 * y]), sl2, -lq.x)),
+                        ex2(fmaf(__uint_as_float(sv[4 * y + 1]), sl2, -lq.y)),
+                        ex2(fmaf(__uint_as_float(sv[4 * y + 2]), sl2, -lq.z)),
+                        ex2(fmaf(__uint_as_float(sv[4 * y + 3]), sl2, -lq.w))};
+          if (q0 < diag_lim) {
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               if (q0 + e < diag_lim) p[e] = 0.f;
           }
-          const float g0 = p[0] * (__uint_as_float(dv[4 * x]) - dq.x);
-          const float g1 = p[1] * (__uint_as_float(dv[4 * x + 1]) - dq.y);
-          const float g2 = p[2] * (__uint_as_float(dv[4 * x + 2]) - dq.z);
-          const float g3 = p[3] * (__uint_as_float(dv[4 * x + 3]) - dq.w);
-          pk[2 * x] = pack_bf16x2(p[0], p[1]);
-          pk[2 * x + 1] = pack_bf16x2(p[2], p[3]);
-          dk[2 * x] = pack_bf16x2(g0, g1);
-          dk[2 * x + 1] = pack_bf16x2(g2, g3);
+          const float g0 = p[0] * (__uint_as_float(dv[4 * y]) - dq.x);
+          const float g1 = p[1] * (__uint_as_float(dv[4 * y + 1]) - dq.y);
+          const float g2 = p[2] * (__uint_as_float(dv[4 * y + 2]) - dq.z);
+          const float g3 = p[3] * (__uint_as_float(dv[4 * y + 3]) - dq.w);
+          pk[2 * y] = pack_bf16x2(p[0], p[1]);
+          pk[2 * y + 1] = pack_bf16x2(p[2], p[3]);
+          dk[2 * y] = pack_bf16x2(g0, g1);
+          dk[2 * y + 1] = pack_bf16x2(g2, g3);
         }
-        // P^T chunk -> columns [16c, 16c+16) of this half's dP^T columns
+        // P^T chunk -> columns [16c, 16c+16) of this buffer's dP^T columns
         // (their dP^T values were loaded by this or the previous chunk).
         tmem_st16(tDP + c * 16, pk);
-        // dS^T chunk: local queries [32c, 32c+32) of key row kr, 128-byte swizzled.
+        // dS^T chunk: queries [32c, 32c+32) of key row kr, 128-byte swizzled.
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const uint32_t chunk = static_cast<uint32_t>(c * 4 + u);
-          uint4 val = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ sw) << 4)) = val;
+          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ sw) << 4)) =
+              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
       }
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready[hf]);
+      mbar_arrive(&bars->p_ready[x]);
     }
     // Epilogue: dV_j rows (this thread's key row), half of the columns per warpgroup.
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
       tc_fence_after();
-      const int key = j * kB + kr;
+      const int key = j * kKT + kr;
       __nv_bfloat16* dst = a.dv + (static_cast<size_t>(bkv) * a.N + key) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
-        const int c = hf * (D / 64) + cc;
+        const int c = x * (D / 64) + cc;
         uint32_t vv[32];
         tmem_ld32(tmem + lane_off + C::kColDV + c * 32, vv);
         uint4 o4[4];
@@ -435,58 +436,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kDqWarp0) {
-    // ----------------------------------------------- dQ_i readout (query rows)
+    // ------------------------------------------- dQ_i^T readout (columns of dQ)
     const int quad = warp & 3;
-    const int qr = quad * 32 + lane;
+    const int m = quad * 32 + lane;                        // column of dQ (tensor-memory lane)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tDQ = tmem + lane_off + C::kColDP;
-    uint8_t* stage = smem + C::kOffDS;                     // two 128 x 32 fp32 boxes, 128-byte swizzled
-    const uint32_t sw = static_cast<uint32_t>(qr & 7);
+    uint8_t* stage = smem + C::kOffST;                     // D/32 boxes of 64 rows x 32 fp32, swizzled
     const bool leader = (warp == kDqWarp0 && lane == 0);
     if (leader) tma_prefetch_desc(&tmDQacc);
+    // Element (query q, column m) of the staged tile.
+    uint8_t* col = stage + (m >> 5) * C::kStBox + ((m & 3) << 2);
+    const uint32_t chunk = static_cast<uint32_t>((m & 31) >> 2);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      ok = dq_group_all(wait_bar(&bars->dq_full, it & 1, w));
+      const int x = it & 1;
+      ok = dq_group_all(wait_bar(&bars->dq_full[x], (it >> 1) & 1, w));
       if (!ok) break;
       tc_fence_after();
       const int h = g * r + it / nqi;
       const int i = i0 + it % nqi;
       const int bh = b * a.Hq + h;
-      // The dQ and dK MMAs that read dS^T have completed (dq_full), and the
-      // softmax-gradient warps write dS^T again only after the next dP^T,
-      // which waits for dq_empty: the buffer is this warpgroup's until then.
-#pragma unroll
-      for (int rd = 0; rd < D / 64; ++rd) {
-#pragma unroll
-        for (int bx = 0; bx < 2; ++bx) {
-          uint32_t vv[32];
-          tmem_ld32(tDQ + rd * 64 + bx * 32, vv);
-          uint8_t* row = stage + bx * (kB * 128) + qr * 128;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(row + ((static_cast<uint32_t>(u) ^ sw) << 4)) =
-                make_uint4(vv[4 * u], vv[4 * u + 1], vv[4 * u + 2], vv[4 * u + 3]);
-        }
-        fence_async_smem();
-        dq_group_sync();
-        if (leader) {
-          // Rows past N fall outside the tensor map's row extent and are dropped.
-          tma_reduce_add_3d(&tmDQacc, stage, rd * 64, i * kB, bh);
-          tma_reduce_add_3d(&tmDQacc, stage + kB * 128, rd * 64 + 32, i * kB, bh);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        dq_group_sync();
-      }
+      uint32_t v0[32], v1[32];
+      const uint32_t tDQ = tmem + lane_off + C::kColDP + 64 * x;
+      tmem_ld32(tDQ, v0);
+      tmem_ld32(tDQ + 32, v1);
       tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
+      mbar_arrive(&bars->dq_empty[x]);
+      // The staging tile is free once the previous reduction has read it.
+      if (leader) bulk_wait_read0();
+      dq_group_sync();
+      if (m < D) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          *reinterpret_cast<uint32_t*>(col + q * 128 + ((chunk ^ static_cast<uint32_t>(q & 7)) << 4)) = v0[q];
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          *reinterpret_cast<uint32_t*>(col + (q + 32) * 128 + ((chunk ^ static_cast<uint32_t>(q & 7)) << 4)) =
+              v1[q];
+      }
+      fence_async_smem();
+      dq_group_sync();
+      if (leader) {
+        // Rows past N fall outside the tensor map's row extent and are dropped.
+#pragma unroll
+        for (int bx = 0; bx < D / 32; ++bx) tma_reduce_add_3d(&tmDQacc, stage + bx * C::kStBox, bx * 32, i * kQT, bh);
+        bulk_commit();
+      }
     }
     if (leader) bulk_wait0();
-    // Epilogue: dK_j = scale * accumulated dS^T Q (this thread's key row).
+    // Epilogue: dK_j = scale * accumulated dS^T Q (row m = key row).
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
       tc_fence_after();
-      const int key = j * kB + qr;
+      const int key = j * kKT + m;
       __nv_bfloat16* dst = a.dk + (static_cast<size_t>(bkv) * a.N + key) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -585,7 +586,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   float* dsum = static_cast<float*>(workspace);
   const size_t dsum_bytes = ((static_cast<size_t>(rows) * 4 + 255) / 256) * 256;
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsum_bytes);
-  if (!encode_f32_tile_map(&tdq, dq_acc, s.d, s.N, s.B * s.Hq, 32, kB)) return cudaErrorInvalidValue;
+  if (!encode_f32_tile_map(&tdq, dq_acc, s.d, s.N, s.B * s.Hq, 32, kQT)) return cudaErrorInvalidValue;
 
   bwd_pre_kernel<D><<<grid_for(rows, 8, 148 * 64), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_resid),
@@ -600,15 +601,14 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   BwdArgs a;
   a.lse = lse;
   a.dsum = dsum;
-  a.dq_acc = dq_acc;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.N = s.N;
   a.Hq = s.Hq;
   a.Hkv = s.Hkv;
   a.BHkv = s.B * s.Hkv;
-  a.nk = (s.N + kB - 1) / kB;
-  a.nq = a.nk;
+  a.nk = (s.N + kKT - 1) / kKT;
+  a.nq = (s.N + kQT - 1) / kQT;
   a.scale = s.scale;
   a.scale_log2 = s.scale * kLog2e;
   a.ctl = ctl;
