@@ -11,9 +11,17 @@
 #include "../../include/fa_profile.h"
 #include "../../include/fa_test.h"
 #include "fa_internal.h"
+#include "sm100.cuh"
 
 namespace fa {
 namespace {
+
+__global__ void test_exp2_kernel(const float* x, float* yp, float* ye, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    yp[i] = exp2_poly(x[i]);
+    ye[i] = ex2(x[i]);
+  }
+}
 
 constexpr int kMaxDevices = 64;
 
@@ -252,6 +260,15 @@ void fa_set_watchdog_ns(uint64_t ns) { g_budget_ns.store(ns < 1000000ull ? 10000
 // (1 = the forward producer never loads the first K tile) so that the
 // watchdog path can be exercised without faulting the GPU.
 void fa_test_set_fault(int code) { g_fault.store(code); }
+
+int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* stream) {
+  if (!x || !y_poly || !y_ex2 || n < 0) return FA_ERR_INVALID_ARGUMENT;
+  if (n == 0) return FA_OK;
+  const int blocks = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
+  test_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_ex2, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
 
 void fa_profile_set_bwd_events(void* after_pre, void* after_main) {
   g_ev_pre.store(after_pre);

@@ -56,6 +56,12 @@ constexpr int kMmaWarp = 9;
 // rescale until the max grew by more than a margin) turns that weight into
 // 2^delta, whose bf16 rounding moves O by up to 2^-9 |V| on peaky rows.
 constexpr float kRescaleThreshold = 0.0f;  // log2 units
+// Of every 32 exponentials of a row, this many are evaluated on the FMA pipe
+// (exp2_poly) and the rest on the exponential unit. Measured on B200 at
+// N = 8192, d = 128: 0 of 32 is fastest (4, 8, 12 cost 3%, 8%, 14%): the
+// softmax warps are bound by instruction issue, not by the exponential unit,
+// so the extra FMA-pipe instructions only add issue slots.
+constexpr int kPolyPer32 = 0;
 
 template <int D>
 struct FwdCfg {
@@ -272,53 +278,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[t], j & 1, w));
       if (!ok) break;
       tc_fence_after();
-      float s[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c * 32, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]);
-      }
+      uint32_t sr[kBN];
+      tmem_ld128(tS, sr);
       if (j == n - 1) {
         const int k0 = j * kBN;
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
-          if (k0 + i > lim) s[i] = -CUDART_INF_F;
+          if (k0 + i > lim) sr[i] = __float_as_uint(-CUDART_INF_F);
       }
-      float mx = s[0];
+      // Row max as 8 independent partial maxima of three-input max
+      // instructions (a linear chain would put 127 dependent instructions on
+      // the softmax's critical path).
+      float pm[8];
 #pragma unroll
-      for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, s[i]);
-      const float m_cand = mx * sl2;
+      for (int u = 0; u < 8; ++u) pm[u] = __uint_as_float(sr[u]);
+#pragma unroll
+      for (int i = 8; i < kBN; i += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          pm[u] = fmax3(pm[u], __uint_as_float(sr[i + u]), __uint_as_float(sr[i + 8 + u]));
+      pm[0] = fmax3(pm[0], pm[1], pm[2]);
+      pm[3] = fmax3(pm[3], pm[4], pm[5]);
+      pm[6] = fmaxf(pm[6], pm[7]);
+      const float m_cand = fmax3(pm[0], pm[3], pm[6]) * sl2;
+      // Warp-uniform: rescale O when some row of the warp has a new max.
+      bool rescale = false;
+      float alpha = 1.f;
       if (j == 0) {
         m = m_cand;
       } else if (__any_sync(0xffffffffu, m_cand > m + kRescaleThreshold)) {
         const float m_new = fmaxf(m, m_cand);
-        const float alpha = ex2(m - m_new);
+        alpha = ex2(m - m_new);
         m = m_new;
         l *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t oo[16];
-          tmem_ld16(tO + c * 16, oo);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) oo[i] = __float_as_uint(__uint_as_float(oo[i]) * alpha);
-          tmem_st16(tO + c * 16, oo);
-        }
+        rescale = true;
       }
       const float neg_m = -m;
-      float sum = 0.f;
+      float ps[8];  // 8 independent partial row sums
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(s[c * 32 + 2 * i], sl2, neg_m));
-          const float p1 = ex2(fmaf(s[c * 32 + 2 * i + 1], sl2, neg_m));
-          sum += p0 + p1;
+          const float x0 = fmaf(__uint_as_float(sr[c * 32 + 2 * i]), sl2, neg_m);
+          const float x1 = fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, neg_m);
+          const float p0 = (2 * i < kPolyPer32) ? exp2_poly(x0) : ex2(x0);
+          const float p1 = (2 * i + 1 < kPolyPer32) ? exp2_poly(x1) : ex2(x1);
+          ps[(2 * i) & 7] += p0;
+          ps[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);
+      }
+      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (rescale) {
+        // O holds every earlier product (see the ordering argument above);
+        // scale this row by alpha before P V is added to it.
+        if constexpr (D == 128) {
+          uint32_t ov[128];
+          tmem_ld128(tO, ov);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o32[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(ov[c * 32 + i]) * alpha);
+            tmem_st32(tO + c * 32, o32);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o32[32];
+            tmem_ld32(tO + c * 32, o32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+            tmem_st32(tO + c * 32, o32);
+          }
+        }
       }
       l += sum;
       tmem_st_wait();

@@ -15,11 +15,22 @@
 #ifndef FA_TEST_H_
 #define FA_TEST_H_
 
+#include "fa.h"
+
 #ifdef __cplusplus
 extern "C" {
 #endif
 
 void fa_test_set_fault(int code);
+
+/*
+ * Evaluates, for n device floats x (each <= 0), the forward kernel's
+ * FMA-pipe exponential into y_poly and the exponential unit's ex2.approx
+ * into y_ex2 (device buffers of n floats), asynchronously on `stream`.
+ * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (null pointer, n < 0) or
+ * FA_ERR_CUDA.
+ */
+int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* stream);
 
 #ifdef __cplusplus
 }
