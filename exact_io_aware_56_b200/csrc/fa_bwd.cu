@@ -99,6 +99,7 @@ struct BwdArgs {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Hq, Hkv, BHkv, nk, nq;
+  int group;  // KV heads per scheduling group (see the work-unit comment)
   float scale, scale_log2;
   LaunchCtl ctl;
 };
@@ -165,10 +166,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch, KV head, key tile j); the longest units (smallest j
-  // when causal) get the lowest block indices (longest-processing-time order).
-  const int bkv = blockIdx.x % a.BHkv;
-  const int j = blockIdx.x / a.BHkv;
+  // Work unit: (batch, KV head, key tile j). KV heads are taken in groups
+  // (all of them when causal, where longest-first order matters most;
+  // otherwise small enough that their query heads' Q, dO and dQ-accumulator
+  // tiles stay in L2 while the resident CTAs sweep them); within a group the
+  // longest units (smallest j when causal) come first.
+  const int per_group = a.group * a.nk;
+  const int grp = blockIdx.x / per_group;
+  const int rem = blockIdx.x - grp * per_group;
+  const int gsize = min(a.group, a.BHkv - grp * a.group);
+  const int bkv = grp * a.group + rem % gsize;
+  const int j = rem / gsize;
   const int r = a.Hq / a.Hkv;
   const int b = bkv / a.Hkv;
   const int g = bkv % a.Hkv;
@@ -609,6 +617,9 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.BHkv = s.B * s.Hkv;
   a.nk = (s.N + kKT - 1) / kKT;
   a.nq = (s.N + kQT - 1) / kQT;
+  // Causal units differ in length: keep strict longest-first order over all
+  // KV heads. Non-causal units are equal: group KV heads for L2 locality.
+  a.group = CAUSAL ? a.BHkv : l2_head_group(static_cast<long long>(8) * (s.Hq / s.Hkv) * s.N * D, a.BHkv);
   a.scale = s.scale;
   a.scale_log2 = s.scale * kLog2e;
   a.ctl = ctl;

@@ -85,6 +85,7 @@ struct FwdArgs {
   __nv_bfloat16* o_resid;  // optional: bf16(O - bf16(O)), the rounding residual of o
   float* lse;
   int N, Hq, Hkv, BH, n_pairs, nk;
+  int group;  // heads per scheduling group (see the work-unit comment)
   float scale_log2;
   LaunchCtl ctl;
 };
@@ -112,12 +113,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch*head, pair of Q tiles). The heaviest pairs (largest
-  // query index, most K/V tiles when causal) get the lowest block indices so
-  // they start first (longest-processing-time order); heads sharing a KV
-  // head are adjacent.
-  const int bh = blockIdx.x % a.BH;
-  const int pair = a.n_pairs - 1 - blockIdx.x / a.BH;
+  // Work unit: (batch*head, pair of Q tiles). Heads are taken in groups
+  // (all heads in one group when causal, where longest-first order matters
+  // most; otherwise small enough that a group's K/V tiles stay in L2 while
+  // the resident CTAs stream them); within a group the heaviest pairs
+  // (largest query index, most K/V tiles when causal) come first and heads
+  // sharing a KV head are adjacent.
+  const int per_group = a.group * a.n_pairs;
+  const int grp = blockIdx.x / per_group;
+  const int rem = blockIdx.x - grp * per_group;
+  const int gsize = min(a.group, a.BH - grp * a.group);
+  const int bh = grp * a.group + rem % gsize;
+  const int pair = a.n_pairs - 1 - rem / gsize;
   const int h = bh % a.Hq;
   const int b = bh / a.Hq;
   const int kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
@@ -424,6 +431,9 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.BH = s.B * s.Hq;
   a.nk = (s.N + kBN - 1) / kBN;
   a.n_pairs = (s.N + 2 * kBM - 1) / (2 * kBM);
+  // Causal units differ in length: keep strict longest-first order over all
+  // heads. Non-causal units are equal: group heads for L2 locality.
+  a.group = CAUSAL ? a.BH : l2_head_group(static_cast<long long>(4) * s.N * D / (s.Hq / s.Hkv), a.BH);
   a.scale_log2 = s.scale * 1.4426950408889634f;
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.n_pairs) * a.BH;

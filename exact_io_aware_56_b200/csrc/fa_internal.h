@@ -23,6 +23,17 @@ struct LaunchCtl {
   cudaEvent_t ev_after_main;
 };
 
+// Number of heads to schedule together so that their per-head working set
+// (`bytes_per_head`) stays within a share of L2 that the resident CTAs can
+// keep hot; at least 1, at most `heads`.
+inline int l2_head_group(long long bytes_per_head, int heads) {
+  constexpr long long kBudget = 48ll << 20;
+  long long g = bytes_per_head > 0 ? kBudget / bytes_per_head : heads;
+  if (g < 1) g = 1;
+  if (g > heads) g = heads;
+  return static_cast<int>(g);
+}
+
 // Encodes a 3-D bf16 tensor map over [outer][rows][cols] with a box of
 // 64 columns x box_rows rows and 128-byte swizzle. Returns false on failure.
 bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_rows);
