@@ -26,9 +26,9 @@
 //               dV_j += P^T dO_i          (P^T read from tensor memory)
 //               dK_j += dS^T Q_i          (dS^T from shared memory)
 //               dQ_i^T = K_j^T dS_i^T     (M = d: one thread per column of dQ)
-//             dQ_i is staged in shared memory and added to the fp32
-//             accumulator by TMA bulk reductions, which overlap the next
-//             tiles. dK_j (times scale) and dV_j are written once.
+//             dQ_i is added to the fp32 accumulator by coalesced reductions
+//             issued from registers, which overlap the next tiles.
+//             dK_j (times scale) and dV_j are written once.
 //   bwd_post  dq = bf16(scale * accumulator).
 //
 // Warp roles of bwd_main (512 threads):
@@ -41,7 +41,7 @@
 //   warp 9      tensor-memory owner and MMA issuer.
 //   warps 10-11 idle (keep the third warpgroup whole).
 //   warps 12-15 dQ warpgroup: thread = column c of dQ; reads dQ_i^T out of
-//               tensor memory, stages it and issues the bulk reductions;
+//               tensor memory, releases it and issues the reductions;
 //               epilogue stores dK.
 // Tensor memory (512 columns): S^T[2] (64 each) | dP^T[2] (64 each; P^T in
 // bf16 over its first 32 columns, then dQ_i^T over all 64) | dV (D) | dK (D).
@@ -75,15 +75,12 @@ struct BwdCfg {
   static constexpr int kQBox = kQT * 128;                  // one 64-column box of a 64-row tile
   static constexpr int kQTile = kQBox * (D / 64);          // Q_i or dO_i
   static constexpr int kDSTile = kKT * kQT * 2;            // dS^T: 128 keys x 64 queries bf16 (one box)
-  static constexpr int kStBox = kQT * 128;                 // staging: 64 rows x 32 fp32
-  static constexpr int kStTile = kStBox * (D / 32);        // dQ_i fp32, 64 x D
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kKTile;
   static constexpr int kOffQ = kOffV + kKTile;
   static constexpr int kOffDO = kOffQ + kQStages * kQTile;
   static constexpr int kOffDS = kOffDO + kQStages * kQTile;
-  static constexpr int kOffST = kOffDS + 2 * kDSTile;
-  static constexpr int kOffLD = kOffST + kStTile;          // [stage] L2[64], D[64]
+  static constexpr int kOffLD = kOffDS + 2 * kDSTile;      // [stage] L2[64], D[64]
   static constexpr int kOffBar = kOffLD + kQStages * 2 * kQT * 4;
   static constexpr int kUsed = kOffBar + 256;
   static constexpr int kSmemBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
@@ -96,6 +93,7 @@ struct BwdCfg {
 struct BwdArgs {
   const float* lse;
   const float* dsum;    // D_i, fp32 [B*Hq*N]
+  float* dq_acc;        // fp32 [B*Hq*N*d]
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Hq, Hkv, BHkv, nk, nq;
@@ -117,39 +115,15 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// out[tile at (c0, c1, c2)] += smem tile, fp32 add, as one bulk operation.
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(m),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void dq_group_sync() {  // the 128 threads of the dQ warpgroup
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-// AND of `v` over the 128 threads of the dQ warpgroup (also a barrier), so
-// that the four warps always take the same branch around dq_group_sync.
-__device__ __forceinline__ bool dq_group_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return r != 0;
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmDQacc, const BwdArgs a) {
+                    const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -445,19 +419,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------- dQ_i^T readout (columns of dQ)
+    // Lane m of the four warps holds column m of dQ_i for the 64 query rows,
+    // so for each row the 32 lanes of a warp cover 32 consecutive floats: one
+    // fully coalesced 128-byte reduction per warp instruction, straight from
+    // registers (no shared-memory staging, which would compete with the MMA
+    // operand reads for shared-memory bandwidth).
     const int quad = warp & 3;
     const int m = quad * 32 + lane;                        // column of dQ (tensor-memory lane)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    uint8_t* stage = smem + C::kOffST;                     // D/32 boxes of 64 rows x 32 fp32, swizzled
-    const bool leader = (warp == kDqWarp0 && lane == 0);
-    if (leader) tma_prefetch_desc(&tmDQacc);
-    // Element (query q, column m) of the staged tile.
-    uint8_t* col = stage + (m >> 5) * C::kStBox + ((m & 3) << 2);
-    const uint32_t chunk = static_cast<uint32_t>((m & 31) >> 2);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int x = it & 1;
-      ok = dq_group_all(wait_bar(&bars->dq_full[x], (it >> 1) & 1, w));
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->dq_full[x], (it >> 1) & 1, w));
       if (!ok) break;
       tc_fence_after();
       const int h = g * r + it / nqi;
@@ -469,28 +442,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tDQ + 32, v1);
       tc_fence_before();
       mbar_arrive(&bars->dq_empty[x]);
-      // The staging tile is free once the previous reduction has read it.
-      if (leader) bulk_wait_read0();
-      dq_group_sync();
       if (m < D) {
+        const int row0 = i * kQT;
+        float* col = a.dq_acc + (static_cast<size_t>(bh) * a.N + row0) * D + m;
+        const int rows = min(kQT, a.N - row0);
+        if (rows == kQT) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          *reinterpret_cast<uint32_t*>(col + q * 128 + ((chunk ^ static_cast<uint32_t>(q & 7)) << 4)) = v0[q];
+          for (int q = 0; q < 32; ++q) red_add_f32(col + static_cast<size_t>(q) * D, __uint_as_float(v0[q]));
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          *reinterpret_cast<uint32_t*>(col + (q + 32) * 128 + ((chunk ^ static_cast<uint32_t>(q & 7)) << 4)) =
-              v1[q];
-      }
-      fence_async_smem();
-      dq_group_sync();
-      if (leader) {
-        // Rows past N fall outside the tensor map's row extent and are dropped.
+          for (int q = 0; q < 32; ++q) red_add_f32(col + static_cast<size_t>(q + 32) * D, __uint_as_float(v1[q]));
+        } else {
 #pragma unroll
-        for (int bx = 0; bx < D / 32; ++bx) tma_reduce_add_3d(&tmDQacc, stage + bx * C::kStBox, bx * 32, i * kQT, bh);
-        bulk_commit();
+          for (int q = 0; q < 32; ++q)
+            if (q < rows) red_add_f32(col + static_cast<size_t>(q) * D, __uint_as_float(v0[q]));
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (q + 32 < rows) red_add_f32(col + static_cast<size_t>(q + 32) * D, __uint_as_float(v1[q]));
+        }
       }
     }
-    if (leader) bulk_wait0();
     // Epilogue: dK_j = scale * accumulated dS^T Q (row m = key row).
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
@@ -589,12 +559,10 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
                          const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
                          cudaStream_t stream) {
   using C = BwdCfg<D>;
-  CUtensorMap tdq;
   const long long rows = static_cast<long long>(s.B) * s.Hq * s.N;
   float* dsum = static_cast<float*>(workspace);
   const size_t dsum_bytes = ((static_cast<size_t>(rows) * 4 + 255) / 256) * 256;
   float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsum_bytes);
-  if (!encode_f32_tile_map(&tdq, dq_acc, s.d, s.N, s.B * s.Hq, 32, kQT)) return cudaErrorInvalidValue;
 
   bwd_pre_kernel<D><<<grid_for(rows, 8, 148 * 64), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_resid),
@@ -609,6 +577,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   BwdArgs a;
   a.lse = lse;
   a.dsum = dsum;
+  a.dq_acc = dq_acc;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.N = s.N;
@@ -625,7 +594,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.nk) * a.BHkv;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ctl.ev_after_main && (e = cudaEventRecord(ctl.ev_after_main, stream)) != cudaSuccess) return e;
