@@ -19,6 +19,11 @@ notes):
 * The softmax scale multiplies Q K^T before the mask and the softmax.
 * Causal masking hides key j from query i when j > i (queries and keys have
   the same length, so top-left and bottom-right alignment agree).
+* Sliding-window and prefix-LM masks ("FlashAttention: IO-aware exact
+  attention", "The honest limits": separate implementations, not a flag)
+  are read as: key j is visible to query i iff (j <= i and i - j <= window)
+  or j < prefix. window = None means no window (plain causal); prefix = 0
+  means no prefix. Every row then sees at least its own key.
 * Grouped-query attention (the "PREFILL PATH" diagram's notes on decode and
   the explainer's "Use with GQA") groups query heads contiguously: query head
   h reads KV head h // (Hq // Hkv).
@@ -57,15 +62,32 @@ def _check(q, k, v):
     return B, Hq, k.shape[1], N, d
 
 
-def _scores(qrows, kmat, scale, causal, row_ids):
+def visible(row_ids, col_ids, causal, window=None, prefix=0):
+    """Boolean [rows, cols] visibility of keys to queries (see module docstring)."""
+    r = np.asarray(row_ids)[:, None]
+    c = np.asarray(col_ids)[None, :]
+    if not causal and window is None and prefix == 0:
+        return np.ones((r.shape[0], c.shape[1]), dtype=bool)
+    vis = c <= r
+    if window is not None:
+        vis &= (r - c) <= window
+    if prefix:
+        vis |= c < prefix
+    return vis
+
+
+def _masked(causal, window, prefix):
+    return causal or window is not None or prefix > 0
+
+
+def _scores(qrows, kmat, scale, causal, row_ids, window=None, prefix=0):
     """Rows of S = scale * Q K^T, with masked entries set to -inf.
 
-    ``row_ids`` are the query positions of ``qrows`` (used by the causal mask).
+    ``row_ids`` are the query positions of ``qrows`` (used by the masks).
     """
     S = scale * (qrows @ kmat.T)
-    if causal:
-        cols = np.arange(kmat.shape[0])
-        S[cols[None, :] > np.asarray(row_ids)[:, None]] = -np.inf
+    if _masked(causal, window, prefix):
+        S[~visible(row_ids, np.arange(kmat.shape[0]), True, window, prefix)] = -np.inf
     return S
 
 
@@ -80,7 +102,7 @@ def _softmax_rows(S):
     return E / l, (m + np.log(l))[:, 0]
 
 
-def attn_fwd_ref(q, k, v, causal: bool, scale: float):
+def attn_fwd_ref(q, k, v, causal: bool, scale: float, window=None, prefix=0):
     """Naive forward: S and P materialised, two-pass softmax, O = P V.
 
     FlashAttention: IO-aware exact attention, "NAIVE" box of the "NAIVE
@@ -97,7 +119,7 @@ def attn_fwd_ref(q, k, v, causal: bool, scale: float):
             g = kv_head_of(h, Hq, Hkv)
             for r0 in range(0, N, _ROW_CHUNK):
                 rows = np.arange(r0, min(N, r0 + _ROW_CHUNK))
-                S = _scores(q[b, h, rows], k[b, g], scale, causal, rows)
+                S = _scores(q[b, h, rows], k[b, g], scale, causal, rows, window, prefix)
                 P, Lr = _softmax_rows(S)
                 O[b, h, rows] = P @ v[b, g]
                 L[b, h, rows] = Lr
@@ -105,7 +127,7 @@ def attn_fwd_ref(q, k, v, causal: bool, scale: float):
 
 
 def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
-                        block_q: int = 128, block_k: int = 128):
+                        block_q: int = 128, block_k: int = 128, window=None, prefix=0):
     """Tiled forward with the online softmax, in the pages' order.
 
     FlashAttention: IO-aware exact attention, "FLASH" box of the "NAIVE
@@ -135,8 +157,8 @@ def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
                 for j0 in range(0, N, block_k):
                     cols = np.arange(j0, min(N, j0 + block_k))
                     S = scale * (Qb @ k[b, g, cols].T)
-                    if causal:
-                        S[cols[None, :] > rows[:, None]] = -np.inf
+                    if _masked(causal, window, prefix):
+                        S[~visible(rows, cols, True, window, prefix)] = -np.inf
                     m_new = np.maximum(m, S.max(axis=1))
                     # A row whose blocks so far are all masked keeps m = -inf;
                     # its factors are then defined as 1 (nothing to rescale).
@@ -151,7 +173,7 @@ def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
     return O_out, L_out
 
 
-def attn_bwd_ref(q, k, v, dout, causal: bool, scale: float):
+def attn_bwd_ref(q, k, v, dout, causal: bool, scale: float, window=None, prefix=0):
     """Gradients of sum(dout * O) with respect to q, k, v.
 
     The pages state only that the backward pass rebuilds P from Q, K and L
@@ -174,7 +196,7 @@ def attn_bwd_ref(q, k, v, dout, causal: bool, scale: float):
             g = kv_head_of(h, Hq, Hkv)
             for r0 in range(0, N, _ROW_CHUNK):
                 rows = np.arange(r0, min(N, r0 + _ROW_CHUNK))
-                S = _scores(q[b, h, rows], k[b, g], scale, causal, rows)
+                S = _scores(q[b, h, rows], k[b, g], scale, causal, rows, window, prefix)
                 P, _ = _softmax_rows(S)
                 dO = dout[b, h, rows]
                 dv[b, g] += P.T @ dO
@@ -186,7 +208,7 @@ def attn_bwd_ref(q, k, v, dout, causal: bool, scale: float):
     return dq, dk, dv
 
 
-def attn_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
+def attn_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows, window=None, prefix=0):
     """O and L of query head ``h`` of batch ``b`` at the given query rows only.
 
     Same arithmetic as :func:`attn_fwd_ref` restricted to some rows (each row
@@ -200,14 +222,14 @@ def attn_fwd_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
     L = np.empty(len(rows))
     for c0 in range(0, len(rows), _ROW_CHUNK):
         rr = rows[c0:c0 + _ROW_CHUNK]
-        S = _scores(q[b, h, rr], k[b, g], scale, causal, rr)
+        S = _scores(q[b, h, rr], k[b, g], scale, causal, rr, window, prefix)
         P, Lr = _softmax_rows(S)
         O[c0:c0 + len(rr)] = P @ v[b, g]
         L[c0:c0 + len(rr)] = Lr
     return O, L
 
 
-def attn_bwd_rows(q, k, v, dout, causal: bool, scale: float, b: int, h: int, rows):
+def attn_bwd_rows(q, k, v, dout, causal: bool, scale: float, b: int, h: int, rows, window=None, prefix=0):
     """dQ of query head ``h`` of batch ``b`` at the given query rows only.
 
     dQ_i = scale * sum_j P_ij (dP_ij - D_i) K_j needs only row i of P and dP
@@ -219,7 +241,7 @@ def attn_bwd_rows(q, k, v, dout, causal: bool, scale: float, b: int, h: int, row
     dq = np.empty((len(rows), q.shape[3]))
     for c0 in range(0, len(rows), _ROW_CHUNK):
         rr = rows[c0:c0 + _ROW_CHUNK]
-        S = _scores(q[b, h, rr], k[b, g], scale, causal, rr)
+        S = _scores(q[b, h, rr], k[b, g], scale, causal, rr, window, prefix)
         P, _ = _softmax_rows(S)
         dP = dout[b, h, rr] @ v[b, g].T
         D = (P * dP).sum(axis=1, keepdims=True)
@@ -227,7 +249,7 @@ def attn_bwd_rows(q, k, v, dout, causal: bool, scale: float, b: int, h: int, row
     return dq
 
 
-def attn_bwd_kv_rows(q, k, v, dout, causal: bool, scale: float, b: int, g: int, keys):
+def attn_bwd_kv_rows(q, k, v, dout, causal: bool, scale: float, b: int, g: int, keys, window=None, prefix=0):
     """dK and dV of KV head ``g`` of batch ``b`` at the given key rows only.
 
     Column j of P and dS depends on every query row's logsumexp and D_i, so
@@ -243,7 +265,7 @@ def attn_bwd_kv_rows(q, k, v, dout, causal: bool, scale: float, b: int, g: int, 
     for h in range(g * r, (g + 1) * r):
         for r0 in range(0, N, _ROW_CHUNK):
             rows = np.arange(r0, min(N, r0 + _ROW_CHUNK))
-            S = _scores(q[b, h, rows], k[b, g], scale, causal, rows)
+            S = _scores(q[b, h, rows], k[b, g], scale, causal, rows, window, prefix)
             P, _ = _softmax_rows(S)
             dO = dout[b, h, rows]
             dP = dO @ v[b, g].T

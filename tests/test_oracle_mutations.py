@@ -33,7 +33,7 @@ _orig_scores = A._scores
 _orig_softmax = A._softmax_rows
 
 
-def scores_mask_off_by_one(qrows, kmat, scale, causal, row_ids):
+def scores_mask_off_by_one(qrows, kmat, scale, causal, row_ids, window=None, prefix=0):
     S = scale * (qrows @ kmat.T)
     if causal:
         cols = np.arange(kmat.shape[0])
@@ -41,13 +41,13 @@ def scores_mask_off_by_one(qrows, kmat, scale, causal, row_ids):
     return S
 
 
-def scores_no_scale(qrows, kmat, scale, causal, row_ids):
-    return _orig_scores(qrows, kmat, 1.0, causal, row_ids)
+def scores_no_scale(qrows, kmat, scale, causal, row_ids, window=None, prefix=0):
+    return _orig_scores(qrows, kmat, 1.0, causal, row_ids, window, prefix)
 
 
-def scores_transposed(qrows, kmat, scale, causal, row_ids):
+def scores_transposed(qrows, kmat, scale, causal, row_ids, window=None, prefix=0):
     # Uses K's rows in reverse order (a wrong index into K).
-    return _orig_scores(qrows, kmat[::-1], scale, causal, row_ids)
+    return _orig_scores(qrows, kmat[::-1], scale, causal, row_ids, window, prefix)
 
 
 def softmax_unnormalised(S):
