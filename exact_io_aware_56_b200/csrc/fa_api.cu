@@ -144,7 +144,9 @@ using namespace fa;
 extern "C" {
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse, int B,
-                    int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+                    int Hq, int Hkv, int N, int d, int causal, float scale, void* stream, int window = -1,
+                    int prefix = 0) {
+  if (window < -1 || prefix < 0) return FA_ERR_INVALID_ARGUMENT;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(o_resid))
@@ -158,6 +160,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, void* 
       !encode_tile_map(&tv, v, d, N, B * Hkv, 128))
     return FA_ERR_UNSUPPORTED;
   AttnShape s{B, Hq, Hkv, N, d, causal, scale};
+  s.window = window;
+  s.prefix = prefix;
   cudaError_t e = launch_fwd(s, tq, tk, tv, o, o_resid, lse, make_ctl(st), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
@@ -181,7 +185,9 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* o_resid,
                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
-                    int d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+                    int d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream,
+                    int window = -1, int prefix = 0) {
+  if (window < -1 || prefix < 0) return FA_ERR_INVALID_ARGUMENT;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARGUMENT;
   const void* ptrs[] = {q, k, v, o, o_resid, dout, lse, dq, dk, dv, workspace};
   for (const void* p : ptrs)
@@ -189,6 +195,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   int rc = check_shape(B, Hq, Hkv, N, d, causal, scale);
   if (rc != FA_OK) return rc;
   AttnShape s{B, Hq, Hkv, N, d, causal, scale};
+  s.window = window;
+  s.prefix = prefix;
   if (workspace_bytes < bwd_workspace_bytes(s)) return FA_ERR_INVALID_ARGUMENT;
   DevState* st = nullptr;
   if ((rc = device_state(&st)) != FA_OK) return rc;
@@ -216,6 +224,18 @@ int fa_bwd_with_residual(const void* q, const void* k, const void* v, const void
   if (!o_resid) return FA_ERR_INVALID_ARGUMENT;
   return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, workspace,
                   workspace_bytes, stream);
+}
+
+int fa_fwd_masked(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse, int B, int Hq,
+                  int Hkv, int N, int d, int window, int prefix, float scale, void* stream) {
+  return fwd_impl(q, k, v, o, o_resid, lse, B, Hq, Hkv, N, d, 1, scale, stream, window, prefix);
+}
+
+int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* o_resid, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int window,
+                  int prefix, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, 1, scale, workspace,
+                  workspace_bytes, stream, window, prefix);
 }
 
 const char* fa_status_string(int status) {

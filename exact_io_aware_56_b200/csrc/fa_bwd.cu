@@ -98,6 +98,8 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   int N, Hq, Hkv, BHkv, nk, nq;
   int group;  // KV heads per scheduling group (see the work-unit comment)
+  int window;  // left window (a huge value when there is none), mask kind 2
+  int prefix;  // prefix length, mask kind 2
   float scale, scale_log2;
   LaunchCtl ctl;
 };
@@ -119,7 +121,9 @@ __device__ __forceinline__ void red_add_f32(float* addr, float v) {
   asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
-template <int D, bool CAUSAL>
+// MASK: 0 none, 1 causal, 2 causal with a left window and/or a prefix
+// (key j visible to query i iff (j <= i and i - j <= window) or j < prefix).
+template <int D, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -154,8 +158,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = a.Hq / a.Hkv;
   const int b = bkv / a.Hkv;
   const int g = bkv % a.Hkv;
-  const int i0 = CAUSAL ? 2 * j : 0;   // first 64-row query tile that sees key tile j
-  const int nqi = a.nq - i0;           // query tiles per head
+  // Query tiles [i0, i0 + nqi) that see some key of tile j: all of them
+  // without a mask or when the tile holds a prefix key; otherwise from the
+  // tile's first key on (causal) up to its last key plus the window.
+  int i0 = 0, i1 = a.nq;
+  if (MASK == 1) i0 = 2 * j;
+  if (MASK == 2 && j * kKT >= a.prefix) {
+    i0 = 2 * j;
+    const long long last = static_cast<long long>(j) * kKT + kKT - 1 + a.window;
+    i1 = static_cast<int>(min(static_cast<long long>(a.nq), last / kQT + 1));
+  }
+  const int nqi = i1 - i0;             // query tiles per head
   const int n_it = r * nqi;            // (head, query tile) iterations
 
   if (threadIdx.x == 0) {
@@ -349,8 +362,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->dp_full[x], par, w));
       if (!ok) break;
       tc_fence_after();
-      // Local query ql is masked when its position is below this key's.
-      const int diag_lim = CAUSAL ? kKT * j + kr - kQT * i : -1;
+      // Kinds 0, 1: local query ql is masked when its position is below this
+      // key's. Kind 2: the general predicate, unless every pair of the tile
+      // pair is visible (all keys in the prefix, or below every query's
+      // diagonal and inside every query's window).
+      const int diag_lim = MASK == 1 ? kKT * j + kr - kQT * i : -1;
+      const int key = kKT * j + kr;
+      const bool gmask = MASK == 2 && !((kKT * j + kKT <= a.prefix) ||
+                                        (kKT * j + kKT - 1 <= kQT * i && kQT * i + kQT - 1 - kKT * j <= a.window));
 #pragma unroll
       for (int c = 0; c < kQT / 32; ++c) {
         uint32_t sv[32], dv[32];
@@ -370,6 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               if (q0 + e < diag_lim) p[e] = 0.f;
+          }
+          if (gmask) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int qg = kQT * i + q0 + e;
+              if (!((key <= qg && qg - key <= a.window) || key < a.prefix)) p[e] = 0.f;
+            }
           }
           const float g0 = p[0] * (__uint_as_float(dv[4 * y]) - dq.x);
           const float g1 = p[1] * (__uint_as_float(dv[4 * y + 1]) - dq.y);
@@ -553,7 +579,7 @@ int grid_for(long long work, int per_block, int cap) {
   return static_cast<int>(g < cap ? g : cap);
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
                          const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
@@ -571,7 +597,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   if (e != cudaSuccess) return e;
   if (ctl.ev_after_pre && (e = cudaEventRecord(ctl.ev_after_pre, stream)) != cudaSuccess) return e;
 
-  auto kern = bwd_main_kernel<D, CAUSAL>;
+  auto kern = bwd_main_kernel<D, MASK>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   BwdArgs a;
@@ -588,7 +614,9 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.nq = (s.N + kQT - 1) / kQT;
   // Causal units differ in length: keep strict longest-first order over all
   // KV heads. Non-causal units are equal: group KV heads for L2 locality.
-  a.group = CAUSAL ? a.BHkv : l2_head_group(static_cast<long long>(8) * (s.Hq / s.Hkv) * s.N * D, a.BHkv);
+  a.group = MASK == 1 ? a.BHkv : l2_head_group(static_cast<long long>(8) * (s.Hq / s.Hkv) * s.N * D, a.BHkv);
+  a.window = s.window < 0 ? 0x3fffffff : s.window;
+  a.prefix = s.prefix;
   a.scale = s.scale;
   a.scale_log2 = s.scale * kLog2e;
   a.ctl = ctl;
@@ -618,8 +646,14 @@ cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensor
                        const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
                        cudaStream_t stream) {
 #define FA_BWD_ARGS s, tq, tk, tv, tdo, o, o_resid, dout, lse, dq, dk, dv, workspace, ctl, stream
-  if (s.d == 64) return s.causal ? launch_bwd_t<64, true>(FA_BWD_ARGS) : launch_bwd_t<64, false>(FA_BWD_ARGS);
-  return s.causal ? launch_bwd_t<128, true>(FA_BWD_ARGS) : launch_bwd_t<128, false>(FA_BWD_ARGS);
+  switch (s.mask_kind() + (s.d == 64 ? 0 : 3)) {
+    case 0: return launch_bwd_t<64, 0>(FA_BWD_ARGS);
+    case 1: return launch_bwd_t<64, 1>(FA_BWD_ARGS);
+    case 2: return launch_bwd_t<64, 2>(FA_BWD_ARGS);
+    case 3: return launch_bwd_t<128, 0>(FA_BWD_ARGS);
+    case 4: return launch_bwd_t<128, 1>(FA_BWD_ARGS);
+    default: return launch_bwd_t<128, 2>(FA_BWD_ARGS);
+  }
 #undef FA_BWD_ARGS
 }
 

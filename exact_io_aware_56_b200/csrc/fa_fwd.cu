@@ -86,6 +86,8 @@ struct FwdArgs {
   float* lse;
   int N, Hq, Hkv, BH, n_pairs, nk;
   int group;  // heads per scheduling group (see the work-unit comment)
+  int window;  // left window (a huge value when there is none), mask kind 2
+  int prefix;  // prefix length, mask kind 2
   float scale_log2;
   LaunchCtl ctl;
 };
@@ -99,7 +101,13 @@ struct FwdBars {
   int abort;
 };
 
-template <int D, bool CAUSAL>
+// Key j visible to query i under mask kind 2.
+__device__ __forceinline__ bool visible2(int i, int j, int window, int prefix) {
+  return (j <= i && i - j <= window) || j < prefix;
+}
+
+// MASK: 0 none, 1 causal, 2 causal with a left window and/or a prefix.
+template <int D, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -130,8 +138,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
   const int q0 = pair * 2 * kBM;
   int n_t[2];
+  // Mask kind 2: both Q tiles walk one K/V stream, the prefix tiles [0, pre)
+  // then the window tiles [win0, win1): stream position u holds key tile
+  // u < pre ? u : win0 + (u - pre). Tiles in the gap are never visited.
+  int pre = 0, win0 = 0;
+  if (MASK == 2) {
+    const int q_hi = min(q0 + 2 * kBM, a.N) - 1;   // highest real query of the pair
+    pre = min(a.nk, (a.prefix + kBN - 1) / kBN);
+    const int lo_key = (a.window >= q0) ? 0 : q0 - a.window;
+    win0 = max(pre, lo_key / kBN);
+    const int win1 = min(a.nk, q_hi / kBN + 1);
+    n_t[0] = n_t[1] = pre + max(0, win1 - win0);
+  } else {
 #pragma unroll
-  for (int t = 0; t < 2; ++t) n_t[t] = CAUSAL ? min(a.nk, 2 * pair + t + 1) : a.nk;
+    for (int t = 0; t < 2; ++t) n_t[t] = MASK == 1 ? min(a.nk, 2 * pair + t + 1) : a.nk;
+  }
+  auto key_tile = [&](int u) { return (MASK == 2 && u >= pre) ? win0 + (u - pre) : u; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -189,14 +211,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int x = 0; x < C::kBoxes; ++x)
             tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                        j * kBN, kvh);
+                        key_tile(j) * kBN, kvh);
           k_last[s] = u;
         }
         mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
 #pragma unroll
         for (int x = 0; x < C::kBoxes; ++x)
           tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                      j * kBN, kvh);
+                      key_tile(j) * kBN, kvh);
         v_last[s] = u;
       }
       // Every copy issued must land before the CTA may exit.
@@ -277,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_off + 256u + t * D;
     const int n = n_t[t];
     const float sl2 = a.scale_log2;
-    const int lim = CAUSAL ? min(row, a.N - 1) : a.N - 1;  // last visible key
+    const int lim = MASK == 1 ? min(row, a.N - 1) : a.N - 1;  // last visible key (kinds 0, 1)
+    const int qt0 = q0 + t * kBM;                               // first query of this tile
     float m = -CUDART_INF_F;  // running max of scale*log2(e)*s
     float l = 0.f;            // running sum, relative to m
     bool ok = true;
@@ -287,20 +310,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[kBN];
       tmem_ld128(tS, sr);
-      if (j == n - 1) {
-        const int k0 = j * kBN;
+      if (MASK != 2) {
+        if (j == n - 1) {
+          const int k0 = j * kBN;
 #pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (k0 + i > lim) sr[i] = __float_as_uint(-CUDART_INF_F);
+          for (int i = 0; i < kBN; ++i)
+            if (k0 + i > lim) sr[i] = __float_as_uint(-CUDART_INF_F);
+        }
+      } else {
+        const int k0 = key_tile(j) * kBN;
+        // Tile visible to every row of this Q tile: all inside the prefix, or
+        // below every row's diagonal and inside every row's window.
+        const bool full = (k0 + kBN <= a.N) &&
+                          ((k0 + kBN <= a.prefix) || (k0 + kBN - 1 <= qt0 && qt0 + kBM - 1 - k0 <= a.window));
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            if (k0 + i >= a.N || !visible2(row, k0 + i, a.window, a.prefix)) sr[i] = __float_as_uint(-CUDART_INF_F);
+        }
       }
       // Row max as 8 independent partial maxima of three-input max
       // instructions (a linear chain would put 127 dependent instructions on
       // the softmax's critical path).
+      static_assert(kBN % 16 == 0, "the partial maxima take 16 columns per step");
       float pm[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) pm[u] = __uint_as_float(sr[u]);
+      for (int u = 0; u < 8; ++u) pm[u] = fmaxf(__uint_as_float(sr[u]), __uint_as_float(sr[8 + u]));
 #pragma unroll
-      for (int i = 8; i < kBN; i += 16)
+      for (int i = 16; i < kBN; i += 16)
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           pm[u] = fmax3(pm[u], __uint_as_float(sr[i + u]), __uint_as_float(sr[i + 8 + u]));
@@ -312,15 +349,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool rescale = false;
       float alpha = 1.f;
       if (j == 0) {
-        m = m_cand;
+        m = m_cand;  // -inf for a row with no visible key yet (mask kind 2)
       } else if (__any_sync(0xffffffffu, m_cand > m + kRescaleThreshold)) {
         const float m_new = fmaxf(m, m_cand);
-        alpha = ex2(m - m_new);
+        alpha = (MASK == 2 && m_new == -CUDART_INF_F) ? 1.f : ex2(m - m_new);
         m = m_new;
         l *= alpha;
         rescale = true;
       }
-      const float neg_m = -m;
+      // A row with no visible key so far has m = -inf: its masked scores
+      // must give exp(-inf) = 0, not exp(-inf + inf).
+      const float neg_m = (MASK == 2 && m == -CUDART_INF_F) ? 0.f : -m;
       float ps[8];  // 8 independent partial row sums
 #pragma unroll
       for (int u = 0; u < 8; ++u) ps[u] = 0.f;
@@ -414,11 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  auto kern = fwd_kernel<D, CAUSAL>;
+  auto kern = fwd_kernel<D, MASK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
@@ -433,7 +472,9 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.n_pairs = (s.N + 2 * kBM - 1) / (2 * kBM);
   // Causal units differ in length: keep strict longest-first order over all
   // heads. Non-causal units are equal: group heads for L2 locality.
-  a.group = CAUSAL ? a.BH : l2_head_group(static_cast<long long>(4) * s.N * D / (s.Hq / s.Hkv), a.BH);
+  a.group = MASK == 1 ? a.BH : l2_head_group(static_cast<long long>(4) * s.N * D / (s.Hq / s.Hkv), a.BH);
+  a.window = s.window < 0 ? 0x3fffffff : s.window;
+  a.prefix = s.prefix;
   a.scale_log2 = s.scale * 1.4426950408889634f;
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.n_pairs) * a.BH;
@@ -446,11 +487,16 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
 
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
-  if (s.d == 64)
-    return s.causal ? launch_fwd_t<64, true>(s, tq, tk, tv, o, o_resid, lse, ctl, stream)
-                    : launch_fwd_t<64, false>(s, tq, tk, tv, o, o_resid, lse, ctl, stream);
-  return s.causal ? launch_fwd_t<128, true>(s, tq, tk, tv, o, o_resid, lse, ctl, stream)
-                  : launch_fwd_t<128, false>(s, tq, tk, tv, o, o_resid, lse, ctl, stream);
+#define FA_FWD_ARGS s, tq, tk, tv, o, o_resid, lse, ctl, stream
+  switch (s.mask_kind() + (s.d == 64 ? 0 : 3)) {
+    case 0: return launch_fwd_t<64, 0>(FA_FWD_ARGS);
+    case 1: return launch_fwd_t<64, 1>(FA_FWD_ARGS);
+    case 2: return launch_fwd_t<64, 2>(FA_FWD_ARGS);
+    case 3: return launch_fwd_t<128, 0>(FA_FWD_ARGS);
+    case 4: return launch_fwd_t<128, 1>(FA_FWD_ARGS);
+    default: return launch_fwd_t<128, 2>(FA_FWD_ARGS);
+  }
+#undef FA_FWD_ARGS
 }
 
 }  // namespace fa

@@ -13,6 +13,11 @@ struct AttnShape {
   int B, Hq, Hkv, N, d;
   int causal;
   float scale;
+  int window = -1;  // left window of the causal mask, -1 = none
+  int prefix = 0;   // keys below this index are visible to every query
+  // 0: no mask; 1: causal; 2: causal with a window and/or a prefix
+  // (key j visible to query i iff (j <= i and i - j <= window) or j < prefix).
+  int mask_kind() const { return !causal ? 0 : (window < 0 && prefix == 0 ? 1 : 2); }
 };
 
 struct LaunchCtl {

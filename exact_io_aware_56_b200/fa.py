@@ -50,6 +50,10 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd.restype = i
     L.fa_bwd_with_residual.argtypes = [vp] * 10 + [i, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd_with_residual.restype = i
+    L.fa_fwd_masked.argtypes = [vp] * 6 + [i, i, i, i, i, i, i, f, vp]
+    L.fa_fwd_masked.restype = i
+    L.fa_bwd_masked.argtypes = [vp] * 10 + [i, i, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_bwd_masked.restype = i
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_check_device_error.argtypes = [vp]
@@ -95,18 +99,33 @@ def _shapes(q, k):
     return B, Hq, k.shape[1], N, d
 
 
-def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None, o_resid=None) -> None:
+def _mask_args(causal, window, prefix):
+    if window is None and not prefix:
+        return None
+    if not causal:
+        raise ValueError("window / prefix masks extend the causal mask: pass causal=True")
+    return (-1 if window is None else int(window), int(prefix))
+
+
+def fa_fwd(q, k, v, o, lse, causal: bool, scale: float, stream=None, o_resid=None, window=None,
+           prefix: int = 0) -> None:
     """Forward pass into caller-owned ``o`` [B,Hq,N,d] bf16 and ``lse`` [B,Hq,N] fp32.
 
-    With ``o_resid`` (bf16, like ``o``) this calls ``fa_fwd_with_residual``.
+    With ``o_resid`` (bf16, like ``o``) this calls ``fa_fwd_with_residual``;
+    with a ``window`` or a ``prefix`` (causal only) it calls ``fa_fwd_masked``.
     """
     B, Hq, Hkv, N, d = _shapes(q, k)
     bf = torch.bfloat16
     qa, ka, va, oa = (_check_tensor("q", q, bf, (B, Hq, N, d)), _check_tensor("k", k, bf, (B, Hkv, N, d)),
                       _check_tensor("v", v, bf, (B, Hkv, N, d)), _check_tensor("o", o, bf, (B, Hq, N, d)))
     la = _check_tensor("lse", lse, torch.float32, (B, Hq, N))
+    mask = _mask_args(causal, window, prefix)
     tail = (B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
-    if o_resid is None:
+    if mask is not None:
+        ra = None if o_resid is None else _check_tensor("o_resid", o_resid, bf, (B, Hq, N, d))
+        rc, name = lib().fa_fwd_masked(qa, ka, va, oa, ra, la, B, Hq, Hkv, N, d, *mask, float(scale),
+                                       _stream(stream)), "fa_fwd_masked"
+    elif o_resid is None:
         rc, name = lib().fa_fwd(qa, ka, va, oa, la, *tail), "fa_fwd"
     else:
         ra = _check_tensor("o_resid", o_resid, bf, (B, Hq, N, d))
@@ -120,7 +139,7 @@ def fa_bwd_workspace_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
 
 
 def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, workspace, stream=None,
-           o_resid=None) -> None:
+           o_resid=None, window=None, prefix: int = 0) -> None:
     """Backward pass into caller-owned ``dq``, ``dk``, ``dv`` using ``workspace`` (uint8 CUDA tensor).
 
     With ``o_resid`` (from :func:`fa_fwd`) this calls ``fa_bwd_with_residual``.
@@ -136,8 +155,13 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, worksp
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
     ws_bytes = workspace.numel() * workspace.element_size()
+    mask = _mask_args(causal, window, prefix)
     tail = (B, Hq, Hkv, N, d, int(bool(causal)), float(scale), workspace.data_ptr(), ws_bytes, _stream(stream))
-    if o_resid is None:
+    if mask is not None:
+        ra = None if o_resid is None else _check_tensor("o_resid", o_resid, bf, (B, Hq, N, d))
+        rc, name = lib().fa_bwd_masked(*args[:4], ra, *args[4:], B, Hq, Hkv, N, d, *mask, float(scale),
+                                       workspace.data_ptr(), ws_bytes, _stream(stream)), "fa_bwd_masked"
+    elif o_resid is None:
         rc, name = lib().fa_bwd(*args, *tail), "fa_bwd"
     else:
         ra = _check_tensor("o_resid", o_resid, bf, (B, Hq, N, d))
@@ -166,7 +190,8 @@ def fa_profile_set_bwd_events(after_pre=None, after_main=None) -> None:
 
 # ------------------------------------------------------------ conveniences
 
-def attention_forward(q, k, v, causal: bool, scale: float | None = None, stream=None, residual: bool = False):
+def attention_forward(q, k, v, causal: bool, scale: float | None = None, stream=None, residual: bool = False,
+                      window=None, prefix: int = 0):
     """Allocates ``o`` and ``lse`` with torch and runs :func:`fa_fwd`.
 
     Returns ``(o, lse)``, or ``(o, lse, o_resid)`` when ``residual`` is true.
@@ -176,12 +201,12 @@ def attention_forward(q, k, v, causal: bool, scale: float | None = None, stream=
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     o_resid = torch.empty_like(q) if residual else None
-    fa_fwd(q, k, v, o, lse, causal, scale, stream, o_resid=o_resid)
+    fa_fwd(q, k, v, o, lse, causal, scale, stream, o_resid=o_resid, window=window, prefix=prefix)
     return (o, lse, o_resid) if residual else (o, lse)
 
 
 def attention_backward(q, k, v, o, dout, lse, causal: bool, scale: float | None = None, workspace=None,
-                       stream=None, o_resid=None):
+                       stream=None, o_resid=None, window=None, prefix: int = 0):
     """Allocates ``dq``, ``dk``, ``dv`` (and the workspace if not given) and runs :func:`fa_bwd`."""
     B, Hq, Hkv, N, d = _shapes(q, k)
     scale = d ** -0.5 if scale is None else scale
@@ -190,5 +215,6 @@ def attention_backward(q, k, v, o, dout, lse, causal: bool, scale: float | None 
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
-    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace, stream, o_resid=o_resid)
+    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace, stream, o_resid=o_resid, window=window,
+           prefix=prefix)
     return dq, dk, dv

@@ -154,6 +154,28 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                    void* stream);
 
+/*
+ * Masked forward and backward: causal attention restricted by a sliding
+ * window and/or opened by a prefix. Key j is visible to query i iff
+ *     (j <= i and i - j <= window) or j < prefix,
+ * so every query sees at least its own key. window = -1 means no window
+ * (plain causal); window = 0 lets each query see only itself. prefix = 0
+ * means no prefix; prefix >= N gives full (bidirectional) attention. This is
+ * the sliding-window / prefix-LM family that "FlashAttention: IO-aware exact
+ * attention" ("The honest limits") lists as needing its own kernels; here it
+ * is one kernel variant that visits only the key tiles a query tile can see
+ * (the prefix tiles and the window tiles, skipping any gap between them).
+ * Arguments as fa_fwd_with_residual / fa_bwd_with_residual, with the causal
+ * flag replaced by (window, prefix); o_resid may be NULL in both (the
+ * backward then forms D from o alone). FA_ERR_INVALID_ARGUMENT when
+ * window < -1 or prefix < 0.
+ */
+int fa_fwd_masked(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse, int B, int Hq,
+                  int Hkv, int N, int d, int window, int prefix, float scale, void* stream);
+int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* o_resid, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int window,
+                  int prefix, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static text for a status code (for FA_ERR_CUDA: the last CUDA error seen by
  * this thread). Never NULL. */
 const char* fa_status_string(int status);
