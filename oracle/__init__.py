@@ -30,6 +30,8 @@ from .attention import (  # noqa: F401
     attn_fwd_rows,
     attn_bwd_rows,
     attn_bwd_kv_rows,
+    attn_decode_ref,
+    visible,
     kv_head_of,
 )
 from .memory import (  # noqa: F401

@@ -274,3 +274,35 @@ def attn_bwd_kv_rows(q, k, v, dout, causal: bool, scale: float, b: int, g: int, 
             dv += P[:, keys].T @ dO
             dk += scale * (dS[:, keys].T @ q[b, h, rows])
     return dk, dv
+
+
+def attn_decode_ref(q, k, v, scale: float, causal: bool = True):
+    """Decode / short-query attention: Nq new queries against an Nk-key cache.
+
+    FlashAttention: IO-aware exact attention, "PREFILL PATH" diagram (after
+    the prefill "decode loop starts (1 token at a time, now bound by
+    KV-cache bandwidth ...)") and "Two notes" (decode reads the KV cache).
+    The same definition as :func:`attn_fwd_ref` with ``q`` of shape
+    [B, Hq, Nq, d] and ``k``, ``v`` of shape [B, Hkv, Nk, d], Nq <= Nk.
+    Reading taken: the new queries are the last Nq positions of the
+    sequence, so query i sits at position Nk - Nq + i and, when causal, sees
+    keys j <= Nk - Nq + i (bottom-right alignment). Nq = 1 sees every key.
+    Returns ``(O [B, Hq, Nq, d], L [B, Hq, Nq])``.
+    """
+    if q.ndim != 4 or k.ndim != 4 or v.shape != k.shape:
+        raise ValueError("q must be [B, Hq, Nq, d]; k and v [B, Hkv, Nk, d]")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != d or Hq % Hkv != 0 or Nq > Nk:
+        raise ValueError("shapes do not match (need Nq <= Nk and Hq a multiple of Hkv)")
+    O = np.empty((B, Hq, Nq, d))
+    L = np.empty((B, Hq, Nq))
+    pos = np.arange(Nk - Nq, Nk)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            S = _scores(q[b, h], k[b, g], scale, causal, pos)
+            P, Lr = _softmax_rows(S)
+            O[b, h] = P @ v[b, g]
+            L[b, h] = Lr
+    return O, L
