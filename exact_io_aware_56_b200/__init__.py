@@ -6,6 +6,17 @@ thin ctypes binding with the same entry-point names; it raises if the library
 is missing or no CUDA device is present, and there is no CPU fallback.
 """
 
-from .inputs import WORKLOADS, Workload, make_inputs, sample_rows, to_f64, workload_inputs  # noqa: F401
+from .inputs import (  # noqa: F401
+    DECODE_WORKLOADS,
+    WORKLOADS,
+    DecodeWorkload,
+    Workload,
+    make_decode_inputs,
+    make_inputs,
+    sample_rows,
+    to_f64,
+    workload_inputs,
+)
 
-__all__ = ["WORKLOADS", "Workload", "make_inputs", "sample_rows", "to_f64", "workload_inputs"]
+__all__ = ["DECODE_WORKLOADS", "WORKLOADS", "DecodeWorkload", "Workload", "make_decode_inputs", "make_inputs",
+           "sample_rows", "to_f64", "workload_inputs"]

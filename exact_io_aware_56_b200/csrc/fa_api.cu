@@ -38,6 +38,7 @@ struct DevState {
   std::once_flag once;
   bool supported = false;
   unsigned int* err = nullptr;
+  int sms = 0;
 };
 DevState g_dev[kMaxDevices];
 
@@ -65,6 +66,7 @@ int device_state(DevState** out) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return;
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return;
     if (major != 10 || minor != 0) return;
+    if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || st.sms <= 0) return;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return;
     st.err = static_cast<unsigned int*>(p);
@@ -88,6 +90,21 @@ int check_shape(int B, int Hq, int Hkv, int N, int d, int causal, float scale) {
   const long long bh = static_cast<long long>(B) * Hq;
   if (bh > (1LL << 30)) return FA_ERR_UNSUPPORTED;
   if (bh * N * d >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+int check_decode_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || Nq > Nk) return FA_ERR_INVALID_ARGUMENT;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  // Query rows per KV head and (batch, KV head) pairs stay TMA coordinates;
+  // element counts of the query and cache tensors stay below 2^40.
+  const long long rows = static_cast<long long>(Hq / Hkv) * Nq;
+  const long long bkv = static_cast<long long>(B) * Hkv;
+  if (rows > (1LL << 30) || bkv > (1LL << 30)) return FA_ERR_UNSUPPORTED;
+  if (bkv * rows * d >= (1LL << 40) || bkv * Nk * d >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -236,6 +253,38 @@ int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, co
                   int prefix, float scale, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, o_resid, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, 1, scale, workspace,
                   workspace_bytes, stream, window, prefix);
+}
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  if (check_decode_shape(B, Hq, Hkv, Nq, Nk, d, 0, 1.f) != FA_OK) return 0;
+  DecodeShape s{B, Hq, Hkv, Nq, Nk, d, 0, 1.f};
+  return decode_workspace_bytes(s);
+}
+
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+              int Nk, int d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARGUMENT;
+  const void* ptrs[] = {q, k, v, o, lse, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_INVALID_ARGUMENT;
+  int rc = check_decode_shape(B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  DecodeShape s{B, Hq, Hkv, Nq, Nk, d, causal, scale};
+  if (workspace_bytes < decode_workspace_bytes(s)) return FA_ERR_INVALID_ARGUMENT;
+  DevState* st = nullptr;
+  if ((rc = device_state(&st)) != FA_OK) return rc;
+  const DecodePlan plan = make_decode_plan(s, st->sms);
+  // The partials of this plan must fit the shape's workspace bound.
+  if (static_cast<long long>(plan.G) * plan.MS > plan.W / plan.T + 2LL * plan.G) return FA_ERR_UNSUPPORTED;
+  // Queries as [B*Hkv][R][d] (the query heads of a KV head are adjacent),
+  // boxes of one row chunk; K and V as [B*Hkv][Nk][d], boxes of 128 keys.
+  CUtensorMap tq, tk, tv;
+  if (!encode_tile_map(&tq, q, d, plan.R, B * Hkv, 128 / plan.rho) || !encode_tile_map(&tk, k, d, Nk, B * Hkv, 128) ||
+      !encode_tile_map(&tv, v, d, Nk, B * Hkv, 128))
+    return FA_ERR_UNSUPPORTED;
+  cudaError_t e =
+      launch_decode(s, plan, tq, tk, tv, o, lse, workspace, make_ctl(st), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
 
 const char* fa_status_string(int status) {

@@ -58,4 +58,43 @@ cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensor
                        const float* lse, void* dq,
                        void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream);
 
+// Decode / short-query attention: Nq queries per head against an Nk-key
+// cache, queries at the last Nq positions.
+struct DecodeShape {
+  int B, Hq, Hkv, Nq, Nk, d;
+  int causal;
+  float scale;
+};
+
+// At most this many CTAs run the decode kernel (one per SM up to here); the
+// workspace bound below depends on it.
+constexpr int kDecodeMaxCtas = 256;
+
+// Stream-K partition of the decode work. Units are (batch, KV head, chunk of
+// 128/rho query rows) with T key tiles of 128 keys each; the W = units * T
+// tiles, in unit order, are cut into G contiguous runs of nearly equal
+// length, run c being tiles [lo(c), lo(c+1)). A run touches at most MS units.
+struct DecodePlan {
+  long long W;
+  int T, G, MS;
+  int R;         // query rows per KV head: (Hq / Hkv) * Nq
+  int rho;       // replication of the chunk's rows over the 128 lanes (4, 2 or 1)
+  int rv;        // stored rows per copy and partial: min(128 / rho, R)
+  int n_chunks;  // row chunks per KV head
+  __host__ __device__ long long lo(long long c) const { return c * W / G; }
+  // The run holding tile t: the largest c with lo(c) <= t.
+  __host__ __device__ int cta_of(long long t) const { return static_cast<int>(((t + 1) * G + W - 1) / W) - 1; }
+};
+
+DecodePlan make_decode_plan(const DecodeShape& s, int num_ctas);
+
+// Workspace for any plan of this shape with G <= kDecodeMaxCtas: partial O
+// (fp32, d per row) and logsumexp for (units + 2 * G) partials of rho * rv rows
+// (G * MS <= W / T + 2 G).
+size_t decode_workspace_bytes(const DecodeShape& s);
+
+cudaError_t launch_decode(const DecodeShape& s, const DecodePlan& plan, const CUtensorMap& tq,
+                          const CUtensorMap& tk, const CUtensorMap& tv, void* o, float* lse, void* workspace,
+                          const LaunchCtl& ctl, cudaStream_t stream);
+
 }  // namespace fa

@@ -54,6 +54,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_masked.restype = i
     L.fa_bwd_masked.argtypes = [vp] * 10 + [i, i, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd_masked.restype = i
+    L.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    L.fa_decode_workspace_bytes.restype = sz
+    L.fa_decode.argtypes = [vp] * 5 + [i, i, i, i, i, i, i, f, vp, sz, vp]
+    L.fa_decode.restype = i
     L.fa_status_string.argtypes = [i]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_check_device_error.argtypes = [vp]
@@ -170,6 +174,31 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, worksp
         raise FaError(rc, name)
 
 
+def fa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int) -> int:
+    return int(lib().fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_decode(q, k, v, o, lse, causal: bool, scale: float, workspace, stream=None) -> None:
+    """Decode attention: ``q``, ``o`` [B,Hq,Nq,d] bf16 against the cache ``k``, ``v``
+    [B,Hkv,Nk,d] bf16 (Nq <= Nk, queries at the last Nq positions); ``lse``
+    [B,Hq,Nq] fp32; ``workspace`` a uint8 CUDA tensor of at least
+    :func:`fa_decode_workspace_bytes` bytes."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B, Hq, Nq, d] and k [B, Hkv, Nk, d]")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    bf = torch.bfloat16
+    args = [_check_tensor("q", q, bf, (B, Hq, Nq, d)), _check_tensor("k", k, bf, (B, Hkv, Nk, d)),
+            _check_tensor("v", v, bf, (B, Hkv, Nk, d)), _check_tensor("o", o, bf, (B, Hq, Nq, d)),
+            _check_tensor("lse", lse, torch.float32, (B, Hq, Nq))]
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    rc = lib().fa_decode(*args, B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale), workspace.data_ptr(),
+                         workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_decode")
+
+
 def fa_check_device_error(stream=None) -> int:
     return int(lib().fa_check_device_error(_stream(stream)))
 
@@ -218,3 +247,20 @@ def attention_backward(q, k, v, o, dout, lse, causal: bool, scale: float | None 
     fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal, scale, workspace, stream, o_resid=o_resid, window=window,
            prefix=prefix)
     return dq, dk, dv
+
+
+def attention_decode(q, k, v, causal: bool = True, scale: float | None = None, workspace=None, stream=None):
+    """Allocates ``o``, ``lse`` (and the workspace if not given) and runs :func:`fa_decode`.
+
+    Returns ``(o, lse)``.
+    """
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    scale = d ** -0.5 if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(max(16, fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d)), dtype=torch.uint8,
+                                device=q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    fa_decode(q, k, v, o, lse, causal, scale, workspace, stream)
+    return o, lse

@@ -67,6 +67,60 @@ WORKLOADS = {
 }
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Decode against a KV cache: Nq new queries per head, an Nk-key cache.
+
+    Shapes are those of serving a GQA model one token (or a few speculative
+    tokens) at a time; the cache is larger than L2, so every call streams it
+    from HBM.
+    """
+
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def bytes_moved(self) -> int:
+        """Algorithmic HBM bytes of one call: read q, k, v; write o (bf16) and lse (fp32)."""
+        qo = 2 * self.B * self.Hq * self.Nq * self.d * 2
+        kv = 2 * self.B * self.Hkv * self.Nk * self.d * 2
+        return qo + kv + 4 * self.B * self.Hq * self.Nq
+
+    def flops(self) -> float:
+        """Two GEMMs of 2*Nq*Nk*d flops per query head (the causal cut is at most Nq^2/2 keys)."""
+        return 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
+
+
+DECODE_WORKLOADS = {
+    w.name: w
+    for w in [
+        DecodeWorkload("decode_b16_hq32_hkv8_nq1_nk8192_d128", 16, 32, 8, 1, 8192, 128, seed=1100),
+        DecodeWorkload("decode_b4_hq64_hkv8_nq4_nk32768_d128", 4, 64, 8, 4, 32768, 128, seed=1101),
+        DecodeWorkload("decode_b64_hq16_hkv16_nq1_nk2048_d64", 64, 16, 16, 1, 2048, 64, seed=1102),
+    ]
+}
+
+
+def make_decode_inputs(B, Hq, Hkv, Nq, Nk, d, seed):
+    """Draw q [B,Hq,Nq,d] and the cache k, v [B,Hkv,Nk,d] (in that order) as
+    bf16 CPU tensors, i.i.d. standard normals rounded from fp32."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    out = {}
+    for name, shape in (("q", (B, Hq, Nq, d)), ("k", (B, Hkv, Nk, d)), ("v", (B, Hkv, Nk, d))):
+        out[name] = torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
 def make_inputs(B, Hq, Hkv, N, d, seed, qk_gain=1.0, with_dout=True):
     """Draw q, k, v (and dout) as bf16 CPU tensors; see the module docstring."""
     g = torch.Generator(device="cpu").manual_seed(int(seed))

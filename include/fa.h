@@ -176,6 +176,40 @@ int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, co
                   const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int window,
                   int prefix, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Decode / short-query attention against a KV cache.
+ *
+ * Nq new queries per head attend to an Nk-key cache, 1 <= Nq <= Nk. The
+ * queries are the last Nq positions of the sequence: query i sits at
+ * position Nk - Nq + i and, when causal = 1, sees keys j <= Nk - Nq + i
+ * (bottom-right alignment; with Nq = 1 every key is visible either way).
+ * Computes the same O and L as fa_fwd for those rows ("FlashAttention:
+ * IO-aware exact attention", "PREFILL PATH" diagram: the decode loop, one
+ * token at a time, reading the KV cache).
+ *
+ * Layout (bf16 row-major, d contiguous, all device memory owned by the
+ * caller):
+ *   q, o   [B][Hq][Nq][d]      query head h uses KV head h / (Hq/Hkv)
+ *   k, v   [B][Hkv][Nk][d]     the cache
+ *   lse    [B][Hq][Nq] fp32    natural-log row logsumexp
+ * workspace: device memory of at least fa_decode_workspace_bytes(...) bytes,
+ * 16-byte aligned, for the per-split partial results (fp32); its contents
+ * on entry do not matter and are overwritten.
+ *
+ * The cache is split across all SMs (each takes an equal share of the
+ * (batch, KV head) key tiles); partial results are merged by logsumexp in a
+ * second kernel on the same stream. Asynchronous on `stream`. Returns
+ * FA_OK; FA_ERR_INVALID_ARGUMENT for a null or misaligned pointer, a
+ * non-positive size, Nq > Nk, a bad causal flag, a non-finite or
+ * non-positive scale, or a workspace smaller than required;
+ * FA_ERR_UNSUPPORTED for d not 64/128, Hq not a multiple of Hkv, a size
+ * past the index limits, or a device that is not compute capability 10.0;
+ * FA_ERR_CUDA on a launch failure. Nothing is written on an argument error.
+ */
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+              int Nk, int d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static text for a status code (for FA_ERR_CUDA: the last CUDA error seen by
  * this thread). Never NULL. */
 const char* fa_status_string(int status);
