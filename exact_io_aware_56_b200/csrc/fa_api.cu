@@ -32,6 +32,7 @@ std::atomic<uint64_t> g_budget_ns{2000000000ull};
 std::atomic<int> g_fault{0};
 std::atomic<void*> g_ev_pre{nullptr};
 std::atomic<void*> g_ev_main{nullptr};
+std::atomic<void*> g_ev_dec{nullptr};
 thread_local char t_cuda_msg[256] = "no CUDA error recorded";
 
 struct DevState {
@@ -282,8 +283,10 @@ int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (!encode_tile_map(&tq, q, d, plan.R, B * Hkv, 128 / plan.rho) || !encode_tile_map(&tk, k, d, Nk, B * Hkv, 128) ||
       !encode_tile_map(&tv, v, d, Nk, B * Hkv, 128))
     return FA_ERR_UNSUPPORTED;
-  cudaError_t e =
-      launch_decode(s, plan, tq, tk, tv, o, lse, workspace, make_ctl(st), static_cast<cudaStream_t>(stream));
+  LaunchCtl ctl = make_ctl(st);
+  ctl.ev_after_pre = nullptr;
+  ctl.ev_after_main = static_cast<cudaEvent_t>(g_ev_dec.load(std::memory_order_relaxed));
+  cudaError_t e = launch_decode(s, plan, tq, tk, tv, o, lse, workspace, ctl, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
 
@@ -338,6 +341,8 @@ int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* strea
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
+
+void fa_profile_set_decode_event(void* after_main) { g_ev_dec.store(after_main); }
 
 void fa_profile_set_bwd_events(void* after_pre, void* after_main) {
   g_ev_pre.store(after_pre);

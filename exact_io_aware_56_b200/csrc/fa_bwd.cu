@@ -112,6 +112,7 @@ struct BwdBars {
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(BwdBars) <= 256, "barrier block exceeds its shared-memory reservation");
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -34,16 +34,20 @@
 //              S = Q K_j^T (both in shared memory), O += P V_j (P in TMEM).
 //
 // Tensor memory (512 columns allocated):
-//   [0,128) S | [128,192) P (bf16 pairs) | [192,192+D) O_0 | [192+D,192+2D) O_1
-// Copy c writes P only at its own 128/RHO key columns; the rest of its
-// lanes' P columns hold zeros written once at start, so P V sums exactly
-// the copy's keys. Two O buffers let the epilogue of one segment overlap
-// the next segment's MMAs.
+//   [0,256) S_0, S_1 | [256,384) P_0, P_1 (bf16 pairs) | [384,...) O_0 (, O_1)
+// S and P are double-buffered by tile parity, so S_(j+1) runs on the
+// tensor pipe while the softmax turns S_j into P_j. Copy c writes P only
+// at its own 128/RHO key columns; the rest of its lanes' P columns hold
+// zeros written once at start, so P V sums exactly the copy's keys. With
+// two O buffers (d = 64) the epilogue of one segment overlaps the next
+// segment's MMAs.
 //
-// Per tile the MMA thread issues S_j, waits for P_j, issues P_j V_j, so
-// S_(j+1) is issued after P_j V_j; tcgen05 operations complete in issue
-// order, hence once S_(j+1) is complete O holds every earlier product and
-// the softmax may rescale it in place (same argument as the forward).
+// Ordering. The MMA thread issues, per tile j, S_(j+1) and then P_j V_j,
+// so S_(j+1) follows P_(j-1) V_(j-1): once S_(j+1) is complete, the P
+// buffer of parity j+1 is free again. O, however, may still be receiving
+// P_j V_j while the softmax works on tile j+1, so a warp that must rescale
+// O first waits for the pv_done phase of tile j (P_(j+1) V_(j+1) cannot
+// start before this warp hands P_(j+1) back, so that phase is unambiguous).
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -58,13 +62,15 @@ constexpr int kT = 128;  // keys per K/V tile = tensor-memory lanes = Q slots
 constexpr int kDecThreads = 192;
 constexpr int kDecProducer = 4;
 constexpr int kDecMma = 5;
-constexpr uint32_t kColP = 128;
-constexpr uint32_t kColO = 192;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColP = 256;
+constexpr uint32_t kColO = 384;
 
 template <int D>
 struct DecCfg {
   static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kQBufs = (D == 128) ? 1 : 2;
+  static constexpr int kOBufs = (kColO + 2 * D <= 512) ? 2 : 1;
   static constexpr int kBoxBytes = kT * 128;  // 128 rows x 64 bf16 columns
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxBytes * kBoxes;
@@ -75,7 +81,7 @@ struct DecCfg {
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert(kColO + 2 * D <= kTmemCols, "tensor memory budget");
+  static_assert(kColO + kOBufs * D <= kTmemCols, "tensor memory budget");
 };
 
 struct DecArgs {
@@ -90,23 +96,37 @@ struct DecArgs {
 struct DecBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[6], v_full[6], kv_empty[6];
-  uint64_t s_full, p_ready;
+  uint64_t s_full[2], p_ready, pv_done;
   uint64_t o_full[2], o_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(DecBars) <= 256, "barrier block exceeds its shared-memory reservation");
 
-// The j-th segment of this CTA's run: unit u, tiles [j0, j1) of the unit.
-struct Segment {
-  int u, j0, j1;
+// Walks the tiles of this CTA's run [t_lo, t_hi) in order, tracking the
+// unit u, its segment e (0 = the run's first unit) and tile j of the unit
+// without dividing per tile.
+struct TileCursor {
+  long long t, t_hi;
+  int T, u, e, j;
+  __device__ __forceinline__ TileCursor(const DecodePlan& p, long long lo, long long hi) : t(lo), t_hi(hi), T(p.T) {
+    const long long u0 = lo / p.T;
+    u = static_cast<int>(u0);
+    e = 0;
+    j = static_cast<int>(lo - u0 * p.T);
+  }
+  __device__ __forceinline__ bool first(long long lo) const { return t == lo || j == 0; }
+  __device__ __forceinline__ bool last() const { return t == t_hi - 1 || j == T - 1; }
+  __device__ __forceinline__ void next() {
+    ++t;
+    if (++j == T) {
+      j = 0;
+      ++u;
+      ++e;
+    }
+  }
 };
-
-__device__ __forceinline__ Segment segment_of(const DecodePlan& p, long long t_lo, long long t_hi, int e) {
-  const long long u = t_lo / p.T + e;
-  const long long a = max(t_lo, u * p.T), b = min(t_hi, (u + 1) * p.T);
-  return Segment{static_cast<int>(u), static_cast<int>(a - u * p.T), static_cast<int>(b - u * p.T)};
-}
 
 template <int D, int RHO>
 __global__ void __launch_bounds__(kDecThreads, 1)
@@ -115,6 +135,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   using C = DecCfg<D>;
   constexpr int ST = C::kStages;
   constexpr int QB = C::kQBufs;
+  constexpr int OB = C::kOBufs;
   constexpr int RB = kT / RHO;  // rows per unit chunk
   constexpr int CW = kT / RHO;  // key columns per copy
   extern __shared__ uint8_t smem_raw[];
@@ -126,7 +147,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int lane = threadIdx.x & 31;
   const DecodePlan& P = a.plan;
   const long long t_lo = P.lo(blockIdx.x), t_hi = P.lo(blockIdx.x + 1);
-  const int n_seg = static_cast<int>((t_hi - 1) / P.T - t_lo / P.T) + 1;
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -134,14 +154,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_init(&bars->q_empty[b], 1);
       mbar_init(&bars->o_full[b], 1);
       mbar_init(&bars->o_empty[b], kT);
+      mbar_init(&bars->s_full[b], 1);
     }
     for (int s = 0; s < ST; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_ready, kT);
+    mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -155,6 +176,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const Watch w{&bars->abort, a.ctl.err, a.ctl.budget_ns};
+  // The merge kernel may be scheduled now; it waits for this grid's results.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");
 
   if (warp == kDecProducer) {
     // ------------------------------------------------------------ producer
@@ -165,42 +188,37 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       int k_last[ST], q_last[2] = {-1, -1};
 #pragma unroll
       for (int s = 0; s < ST; ++s) k_last[s] = -1;
-      int g = 0;  // tile counter of this CTA
-      bool ok = true;
-      for (int e = 0; ok && e < n_seg; ++e) {
-        const Segment sg = segment_of(P, t_lo, t_hi, e);
-        const int bkv = sg.u / a.n_chunks;
-        const int chunk = sg.u - bkv * a.n_chunks;
-        for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-          const int s = g % ST;
-          const int use = g / ST;
-          if (g >= ST && !(ok = wait_bar(&bars->kv_empty[s], (use - 1) & 1, w))) break;
-          mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+      for (TileCursor ta(P, t_lo, t_hi); ta.t < t_hi; ta.next()) {
+        const int g = static_cast<int>(ta.t - t_lo);
+        const int s = g % ST;
+        const int use = g / ST;
+        const int bkv = ta.u / a.n_chunks;
+        if (g >= ST && !wait_bar(&bars->kv_empty[s], (use - 1) & 1, w)) break;
+        mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+#pragma unroll
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                      ta.j * kT, bkv);
+        mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+#pragma unroll
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
+                      ta.j * kT, bkv);
+        k_last[s] = use;
+        if (ta.first(t_lo)) {
+          // The segment's Q, after its first K/V tile is on its way: RHO
+          // copies of the chunk's RB rows fill the 128 slots.
+          const int qb = ta.e % QB;
+          const int chunk = ta.u - bkv * a.n_chunks;
+          if (ta.e >= QB && !wait_bar(&bars->q_empty[qb], ((ta.e / QB) - 1) & 1, w)) break;
+          mbar_arrive_expect_tx(&bars->q_full[qb], C::kTileBytes);
 #pragma unroll
           for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                        j * kT, bkv);
-          mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
 #pragma unroll
-          for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                        j * kT, bkv);
-          k_last[s] = use;
-          if (j == sg.j0) {
-            // The segment's Q, after its first K/V tile is on its way: RHO
-            // copies of the chunk's RB rows fill the 128 slots.
-            const int qb = e % QB;
-            if (e >= QB && !(ok = wait_bar(&bars->q_empty[qb], ((e / QB) - 1) & 1, w))) break;
-            mbar_arrive_expect_tx(&bars->q_full[qb], C::kTileBytes);
-#pragma unroll
-            for (int x = 0; x < C::kBoxes; ++x)
-#pragma unroll
-              for (int c = 0; c < RHO; ++c)
-                tma_load_3d(&tmQ, &bars->q_full[qb],
-                            smem + C::kOffQ + qb * C::kTileBytes + x * C::kBoxBytes + c * RB * 128, x * 64,
-                            chunk * RB, bkv);
-            q_last[qb] = e / QB;
-          }
+            for (int c = 0; c < RHO; ++c)
+              tma_load_3d(&tmQ, &bars->q_full[qb], smem + C::kOffQ + qb * C::kTileBytes + x * C::kBoxBytes + c * RB * 128,
+                          x * 64, chunk * RB, bkv);
+          q_last[qb] = ta.e / QB;
         }
       }
       // Every copy issued must land before the CTA may exit.
@@ -221,39 +239,58 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const uint32_t sQ = smem_u32(smem + C::kOffQ);
       const uint32_t sK = smem_u32(smem + C::kOffK);
       const uint32_t sV = smem_u32(smem + C::kOffV);
-      int g = 0;
-      bool ok = true;
-      for (int e = 0; ok && e < n_seg; ++e) {
-        const Segment sg = segment_of(P, t_lo, t_hi, e);
-        const int qb = e % QB, ob = e & 1;
-        const uint32_t tO = tmem + kColO + ob * D;
-        if (!(ok = wait_bar(&bars->q_full[qb], (e / QB) & 1, w))) break;
-        if (e >= 2 && !(ok = wait_bar(&bars->o_empty[ob], ((e >> 1) - 1) & 1, w))) break;
-        for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-          const int s = g % ST;
-          const uint32_t par = (g / ST) & 1;
-          if (!(ok = wait_bar(&bars->k_full[s], par, w))) break;
-          tc_fence_after();
-          const uint32_t qa = sQ + qb * C::kTileBytes;
-          const uint32_t ka = sK + s * C::kTileBytes;
+      // S_t = Q K_t^T into S buffer (t - t_lo) & 1.
+      auto issue_s = [&](const TileCursor& ta) -> bool {
+        const int g = static_cast<int>(ta.t - t_lo);
+        const int s = g % ST;
+        const int qb = ta.e % QB;
+        if (ta.first(t_lo) && !wait_bar(&bars->q_full[qb], (ta.e / QB) & 1, w)) return false;
+        if (!wait_bar(&bars->k_full[s], (g / ST) & 1, w)) return false;
+        tc_fence_after();
+        const uint32_t qa = sQ + qb * C::kTileBytes;
+        const uint32_t ka = sK + s * C::kTileBytes;
+        const uint32_t d_s = tmem + kColS + (g & 1) * kT;
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k / 4) * C::kBoxBytes + (k % 4) * 32;
-            mma_ss(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
-          }
-          mma_commit(&bars->s_full);
-          if (!(ok = wait_bar(&bars->p_ready, g & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
-          tc_fence_after();
-          const uint32_t va = sV + s * C::kTileBytes;
-#pragma unroll
-          for (int k = 0; k < kT / 16; ++k)
-            mma_ts(tO, tmem + kColP + k * 8, sdesc_sw128(va + k * 2048, C::kBoxBytes, 1024), idesc_pv,
-                   (j > sg.j0 || k > 0) ? 1u : 0u);
-          mma_commit(&bars->kv_empty[s]);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k / 4) * C::kBoxBytes + (k % 4) * 32;
+          mma_ss(d_s, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
         }
-        if (!ok) break;
-        mma_commit(&bars->o_full[ob]);
-        mma_commit(&bars->q_empty[qb]);
+        mma_commit(&bars->s_full[g & 1]);
+        if (ta.last()) mma_commit(&bars->q_empty[qb]);  // the segment's last read of its Q buffer
+        return true;
+      };
+      // O += P_t V_t.
+      auto issue_pv = [&](const TileCursor& ta) -> bool {
+        const int g = static_cast<int>(ta.t - t_lo);
+        const int s = g % ST;
+        const int ob = ta.e % OB;
+        if (!wait_bar(&bars->p_ready, g & 1, w) || !wait_bar(&bars->v_full[s], (g / ST) & 1, w)) return false;
+        const bool first = ta.first(t_lo);
+        if (first && ta.e >= OB && !wait_bar(&bars->o_empty[ob], ((ta.e / OB) - 1) & 1, w)) return false;
+        tc_fence_after();
+        const uint32_t va = sV + s * C::kTileBytes;
+        const uint32_t d_o = tmem + kColO + ob * D;
+        const uint32_t a_p = tmem + kColP + (g & 1) * 64;
+#pragma unroll
+        for (int k = 0; k < kT / 16; ++k)
+          mma_ts(d_o, a_p + k * 8, sdesc_sw128(va + k * 2048, C::kBoxBytes, 1024), idesc_pv,
+                 (!first || k > 0) ? 1u : 0u);
+        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->pv_done);
+        if (ta.last()) mma_commit(&bars->o_full[ob]);
+        return true;
+      };
+      TileCursor cur(P, t_lo, t_hi), nxt(P, t_lo, t_hi);
+      bool ok = issue_s(nxt);
+      for (nxt.next(); ok && cur.t < t_hi; cur.next(), nxt.next()) {
+        const bool more = nxt.t < t_hi;
+        // With one Q buffer the next segment's Q lands only after this
+        // segment's last S: hand P_t V_t to the tensor pipe before waiting.
+        if (QB == 1 && more && nxt.first(t_lo)) {
+          ok = issue_pv(cur) && issue_s(nxt);
+        } else {
+          ok = (!more || issue_s(nxt)) && issue_pv(cur);
+        }
       }
       // All MMAs issued by this thread must finish before tensor memory is freed.
       mma_commit(&bars->drain);
@@ -265,8 +302,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int cp = slot / RB;           // copy: key columns [cp*CW, cp*CW + CW) of each tile
     const int rr = slot - cp * RB;      // row within the chunk
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off;
-    const uint32_t tP = tmem + lane_off + kColP;
     const float sl2 = a.scale_log2;
     if (RHO > 1) {
       // P columns of the other copies stay zero for the whole kernel.
@@ -274,127 +309,133 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
       for (int i = 0; i < 16; ++i) z[i] = 0u;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st16(tP + c * 16, z);
+      for (int c = 0; c < 8; ++c) tmem_st16(tmem + lane_off + kColP + c * 16, z);
       tmem_st_wait();
     }
     const int RV = min(RB, a.R);
-    int g = 0;
-    bool ok = true;
-    for (int e = 0; ok && e < n_seg; ++e) {
-      const Segment sg = segment_of(P, t_lo, t_hi, e);
-      const int ob = e & 1;
+    float m = -CUDART_INF_F;
+    float l = 0.f;
+    int pos = 0;
+    bool valid = false;
+    for (TileCursor ta(P, t_lo, t_hi); ta.t < t_hi; ta.next()) {
+      const int g = static_cast<int>(ta.t - t_lo);
+      const bool first = ta.first(t_lo);
+      const int ob = ta.e % OB;
+      const uint32_t tS = tmem + lane_off + kColS + (g & 1) * kT;
+      const uint32_t tP = tmem + lane_off + kColP + (g & 1) * 64;
       const uint32_t tO = tmem + lane_off + kColO + ob * D;
-      const int chunk = sg.u % a.n_chunks;
-      const int grow = chunk * RB + rr;  // row within the KV head's R rows
-      const bool valid = rr < RV && grow < a.R;
-      // Last visible key of this row.
-      const int pos = a.causal ? a.Nk - a.Nq + (grow % a.Nq) : a.Nk - 1;
-      float m = -CUDART_INF_F;
-      float l = 0.f;
-      for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-        ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full, g & 1, w));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sr[CW];
-        if constexpr (CW == 128) {
-          tmem_ld128(tS, sr);
-        } else {
-#pragma unroll
-          for (int c = 0; c < CW / 32; ++c) {
-            uint32_t t32[32];
-            tmem_ld32(tS + cp * CW + c * 32, t32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sr[c * 32 + i] = t32[i];
-          }
-        }
-        const int k0 = j * kT + cp * CW;
-        if (k0 + CW - 1 > pos) {
-#pragma unroll
-          for (int i = 0; i < CW; ++i)
-            if (k0 + i > pos) sr[i] = __float_as_uint(-CUDART_INF_F);
-        }
-        float pm[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) pm[u] = fmaxf(__uint_as_float(sr[u]), __uint_as_float(sr[8 + u]));
-#pragma unroll
-        for (int i = 16; i < CW; i += 16)
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            pm[u] = fmax3(pm[u], __uint_as_float(sr[i + u]), __uint_as_float(sr[i + 8 + u]));
-        pm[0] = fmax3(pm[0], pm[1], pm[2]);
-        pm[3] = fmax3(pm[3], pm[4], pm[5]);
-        pm[6] = fmaxf(pm[6], pm[7]);
-        const float m_cand = fmax3(pm[0], pm[3], pm[6]) * sl2;
-        bool rescale = false;
-        float alpha = 1.f;
-        if (j == sg.j0) {
-          m = m_cand;
-        } else if (__any_sync(0xffffffffu, m_cand > m)) {
-          const float m_new = fmaxf(m, m_cand);
-          alpha = (m_new == -CUDART_INF_F) ? 1.f : ex2(m - m_new);
-          m = m_new;
-          l *= alpha;
-          rescale = true;
-        }
-        // A row with no visible key so far keeps m = -inf; its masked
-        // scores must give exp(-inf) = 0, not exp(-inf + inf).
-        const float neg_m = (m == -CUDART_INF_F) ? 0.f : -m;
-        float ps[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+      if (first) {
+        const int chunk = ta.u % a.n_chunks;
+        const int grow = chunk * RB + rr;  // row within the KV head's R rows
+        valid = rr < RV && grow < a.R;
+        pos = a.causal ? a.Nk - a.Nq + (grow % a.Nq) : a.Nk - 1;  // last visible key
+        m = -CUDART_INF_F;
+        l = 0.f;
+      }
+      if (!__all_sync(0xffffffffu, wait_bar(&bars->s_full[g & 1], (g >> 1) & 1, w))) break;
+      tc_fence_after();
+      uint32_t sr[CW];
+      if constexpr (CW == 128) {
+        tmem_ld128(tS, sr);
+      } else {
 #pragma unroll
         for (int c = 0; c < CW / 32; ++c) {
-          uint32_t pk[16];
+          uint32_t t32[32];
+          tmem_ld32(tS + cp * CW + c * 32, t32);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), sl2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, neg_m));
-            ps[(2 * i) & 7] += p0;
-            ps[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tP + cp * (CW / 2) + c * 16, pk);
-        }
-        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        if (rescale) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o32[32];
-            tmem_ld32(tO + c * 32, o32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
-            tmem_st32(tO + c * 32, o32);
-          }
-        }
-        l += sum;
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->p_ready);
-      }
-      if (!ok) break;
-      ok = __all_sync(0xffffffffu, wait_bar(&bars->o_full[ob], (e >> 1) & 1, w));
-      if (!ok) break;
-      tc_fence_after();
-      // Partial of this copy: O / l and logsumexp, or zeros and -inf when
-      // no key of the segment is visible to the row.
-      const long long pidx = static_cast<long long>(blockIdx.x) * P.MS + e;
-      const long long prow = (pidx * RHO + cp) * RV + rr;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t oo[32];
-        tmem_ld32(tO + c * 32, oo);
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * D + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(oo[4 * i]) * inv_l, __uint_as_float(oo[4 * i + 1]) * inv_l,
-                                 __uint_as_float(oo[4 * i + 2]) * inv_l, __uint_as_float(oo[4 * i + 3]) * inv_l);
+          for (int i = 0; i < 32; ++i) sr[c * 32 + i] = t32[i];
         }
       }
-      if (valid) a.part_l[prow] = l > 0.f ? (m + lg2(l)) * 0.69314718055994530942f : -CUDART_INF_F;
+      const int k0 = ta.j * kT + cp * CW;
+      if (k0 + CW - 1 > pos) {
+#pragma unroll
+        for (int i = 0; i < CW; ++i)
+          if (k0 + i > pos) sr[i] = __float_as_uint(-CUDART_INF_F);
+      }
+      float pm[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pm[u] = fmaxf(__uint_as_float(sr[u]), __uint_as_float(sr[8 + u]));
+#pragma unroll
+      for (int i = 16; i < CW; i += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          pm[u] = fmax3(pm[u], __uint_as_float(sr[i + u]), __uint_as_float(sr[i + 8 + u]));
+      pm[0] = fmax3(pm[0], pm[1], pm[2]);
+      pm[3] = fmax3(pm[3], pm[4], pm[5]);
+      pm[6] = fmaxf(pm[6], pm[7]);
+      const float m_cand = fmax3(pm[0], pm[3], pm[6]) * sl2;
+      bool rescale = false;
+      float alpha = 1.f;
+      if (first) {
+        m = m_cand;
+      } else if (__any_sync(0xffffffffu, m_cand > m)) {
+        const float m_new = fmaxf(m, m_cand);
+        alpha = (m_new == -CUDART_INF_F) ? 1.f : ex2(m - m_new);
+        m = m_new;
+        l *= alpha;
+        rescale = true;
+      }
+      // A row with no visible key so far keeps m = -inf; its masked
+      // scores must give exp(-inf) = 0, not exp(-inf + inf).
+      const float neg_m = (m == -CUDART_INF_F) ? 0.f : -m;
+      float ps[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+#pragma unroll
+      for (int c = 0; c < CW / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), sl2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, neg_m));
+          ps[(2 * i) & 7] += p0;
+          ps[(2 * i + 1) & 7] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tP + cp * (CW / 2) + c * 16, pk);
+      }
+      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (rescale) {
+        // O may still be receiving the previous tile's product.
+        if (!__all_sync(0xffffffffu, wait_bar(&bars->pv_done, (g - 1) & 1, w))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o32[32];
+          tmem_ld32(tO + c * 32, o32);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+          tmem_st32(tO + c * 32, o32);
+        }
+      }
+      l += sum;
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->o_empty[ob]);
+      mbar_arrive(&bars->p_ready);
+      if (ta.last()) {
+        if (!__all_sync(0xffffffffu, wait_bar(&bars->o_full[ob], (ta.e / OB) & 1, w))) break;
+        tc_fence_after();
+        // Partial of this copy: O / l and logsumexp, or zeros and -inf when
+        // no key of the segment is visible to the row.
+        const long long pidx = static_cast<long long>(blockIdx.x) * P.MS + ta.e;
+        const long long prow = (pidx * RHO + cp) * RV + rr;
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t oo[32];
+          tmem_ld32(tO + c * 32, oo);
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(a.part_o + prow * D + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(oo[4 * i]) * inv_l, __uint_as_float(oo[4 * i + 1]) * inv_l,
+                                   __uint_as_float(oo[4 * i + 2]) * inv_l, __uint_as_float(oo[4 * i + 3]) * inv_l);
+          }
+        }
+        if (valid) a.part_l[prow] = l > 0.f ? (m + lg2(l)) * 0.69314718055994530942f : -CUDART_INF_F;
+        tc_fence_before();
+        mbar_arrive(&bars->o_empty[ob]);
+      }
     }
   }
 
@@ -408,13 +449,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 }
 
 // Merges each row's partials (every copy of every segment of its unit):
-// one warp per query row, lanes across the head dimension.
+// one warp per query row. Lanes first take one partial each for the max and
+// the sum of e^(L_s - max); the weighted sum of the partial O rows then runs
+// over the head dimension across lanes, four partials per step so their
+// loads overlap. Launched as a programmatic dependent of the decode kernel:
+// it may become resident early and waits for that grid's results here.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_l,
                                                              __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
                                                              const DecodePlan plan, int rows, int R, int rb,
                                                              int rho, int n_chunks) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;  // = bkv * R + grow
@@ -426,29 +472,51 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   const int rv = min(rb, R);
   const long long u = static_cast<long long>(bkv) * n_chunks + chunk;
   const int c0 = plan.cta_of(u * plan.T);
-  const int c1 = plan.cta_of(u * plan.T + plan.T - 1);
+  const int n_parts = (plan.cta_of(u * plan.T + plan.T - 1) - c0 + 1) * rho;
+  // Partial p = (run c0 + p / rho, copy p % rho) -> its row in the workspace.
+  auto prow_of = [&](int p) -> long long {
+    const int c = c0 + p / rho;
+    const long long pidx = static_cast<long long>(c) * plan.MS + (u - plan.lo(c) / plan.T);
+    return (pidx * rho + p % rho) * rv + rr;
+  };
   float mx = -CUDART_INF_F;
-  for (int c = c0; c <= c1; ++c) {
-    const long long pidx = static_cast<long long>(c) * plan.MS + (u - plan.lo(c) / plan.T);
-    for (int cp = 0; cp < rho; ++cp) mx = fmaxf(mx, part_l[(pidx * rho + cp) * rv + rr]);
-  }
+  for (int p = lane; p < n_parts; p += 32) mx = fmaxf(mx, part_l[prow_of(p)]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float den = 0.f;
-  for (int c = c0; c <= c1; ++c) {
-    const long long pidx = static_cast<long long>(c) * plan.MS + (u - plan.lo(c) / plan.T);
-    for (int cp = 0; cp < rho; ++cp) den += expf(part_l[(pidx * rho + cp) * rv + rr] - mx);
-  }
+  for (int p = lane; p < n_parts; p += 32) den += expf(part_l[prow_of(p)] - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
   const float L = mx + logf(den);
   float acc[D / 32];
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
-  for (int c = c0; c <= c1; ++c) {
-    const long long pidx = static_cast<long long>(c) * plan.MS + (u - plan.lo(c) / plan.T);
-    for (int cp = 0; cp < rho; ++cp) {
-      const long long prow = (pidx * rho + cp) * rv + rr;
-      const float wgt = expf(part_l[prow] - L);
-      if (wgt == 0.f) continue;  // also skips rows of segments without a visible key
+  for (int base = 0; base < n_parts; base += 32) {
+    // Lane i holds the weight and row of partial base + i (weight 0 past the
+    // end, and for partials without a visible key, whose L is -inf).
+    const int p = base + lane;
+    float wl = 0.f;
+    long long rl = 0;
+    if (p < n_parts) {
+      rl = prow_of(p);
+      wl = expf(part_l[rl] - L);
+    }
+    const int n = min(32, n_parts - base);
+    for (int i = 0; i < n; i += 4) {
+      float wv[4], x[4][D / 32];
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) acc[i] = fmaf(wgt, part_o[prow * D + i * 32 + lane], acc[i]);
+      for (int q = 0; q < 4; ++q) {
+        wv[q] = __shfl_sync(0xffffffffu, wl, (i + q) & 31);
+        const long long r = __shfl_sync(0xffffffffu, rl, (i + q) & 31);
+        const bool live = i + q < n && wv[q] != 0.f;
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) x[q][k] = live ? part_o[r * D + k * 32 + lane] : 0.f;
+        if (!live) wv[q] = 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) acc[k] = fmaf(wv[q], x[q][k], acc[k]);
     }
   }
 #pragma unroll
@@ -478,11 +546,21 @@ cudaError_t launch_decode_t(const DecodeShape& s, const DecodePlan& plan, const 
   a.ctl = ctl;
   kern<<<plan.G, kDecThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (ctl.ev_after_main && (e = cudaEventRecord(ctl.ev_after_main, stream)) != cudaSuccess) return e;
   const long long rows = static_cast<long long>(s.B) * s.Hkv * plan.R;
-  decode_combine_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(
-      a.part_o, a.part_l, static_cast<__nv_bfloat16*>(o), lse, plan, static_cast<int>(rows), plan.R, kT / RHO,
-      RHO, plan.n_chunks);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, static_cast<const float*>(a.part_o),
+                            static_cast<const float*>(a.part_l), static_cast<__nv_bfloat16*>(o), lse, plan,
+                            static_cast<int>(rows), plan.R, kT / RHO, RHO, plan.n_chunks);
 }
 
 }  // namespace

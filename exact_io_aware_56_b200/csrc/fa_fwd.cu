@@ -100,6 +100,7 @@ struct FwdBars {
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(FwdBars) <= FwdCfg<64>::kBarBytes, "barrier block exceeds its shared-memory reservation");
 
 // Key j visible to query i under mask kind 2.
 __device__ __forceinline__ bool visible2(int i, int j, int window, int prefix) {

@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.fa_test_set_fault.restype = None
     L.fa_profile_set_bwd_events.argtypes = [vp, vp]
     L.fa_profile_set_bwd_events.restype = None
+    L.fa_profile_set_decode_event.argtypes = [vp]
+    L.fa_profile_set_decode_event.restype = None
     _lib = L
     return L
 
@@ -215,6 +217,11 @@ def fa_profile_set_bwd_events(after_pre=None, after_main=None) -> None:
     """Hands two torch.cuda.Event objects (or None) to the timing hook."""
     ptr = lambda e: None if e is None else e.cuda_event
     lib().fa_profile_set_bwd_events(ptr(after_pre), ptr(after_main))
+
+
+def fa_profile_set_decode_event(after_main=None) -> None:
+    """Hands a torch.cuda.Event (or None) to the decode timing hook."""
+    lib().fa_profile_set_decode_event(None if after_main is None else after_main.cuda_event)
 
 
 # ------------------------------------------------------------ conveniences

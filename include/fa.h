@@ -198,7 +198,9 @@ int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, co
  *
  * The cache is split across all SMs (each takes an equal share of the
  * (batch, KV head) key tiles); partial results are merged by logsumexp in a
- * second kernel on the same stream. Asynchronous on `stream`. Returns
+ * second kernel on the same stream (launched as a programmatic dependent of
+ * the first, so it is resident before the first ends). Asynchronous on
+ * `stream`. Returns
  * FA_OK; FA_ERR_INVALID_ARGUMENT for a null or misaligned pointer, a
  * non-positive size, Nq > Nk, a bad causal flag, a non-finite or
  * non-positive scale, or a workspace smaller than required;

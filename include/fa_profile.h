@@ -10,6 +10,11 @@
  * right after the main launch. Passing NULL for both turns the hook off.
  * The setting is process-wide and applies to later fa_bwd calls from any
  * thread; it is meant for benchmarks, not for concurrent production use.
+ *
+ * fa_decode runs two kernels: the split decode kernel and the merge of its
+ * partial results. fa_profile_set_decode_event hands it one event that it
+ * records right after the decode kernel's launch (NULL turns it off), with
+ * the same scope as above.
  */
 #ifndef FA_PROFILE_H_
 #define FA_PROFILE_H_
@@ -19,6 +24,7 @@ extern "C" {
 #endif
 
 void fa_profile_set_bwd_events(void* after_pre, void* after_main);
+void fa_profile_set_decode_event(void* after_main);
 
 #ifdef __cplusplus
 }
