@@ -448,6 +448,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
+// Loads 2 or 4 consecutive floats (8- or 16-byte aligned) into registers.
+__device__ __forceinline__ void load_vec(const float* p, float (&x)[4]) {
+  const float4 t = *reinterpret_cast<const float4*>(p);
+  x[0] = t.x;
+  x[1] = t.y;
+  x[2] = t.z;
+  x[3] = t.w;
+}
+__device__ __forceinline__ void load_vec(const float* p, float (&x)[2]) {
+  const float2 t = *reinterpret_cast<const float2*>(p);
+  x[0] = t.x;
+  x[1] = t.y;
+}
+
 // Merges each row's partials (every copy of every segment of its unit):
 // one warp per query row. Lanes first take one partial each for the max and
 // the sum of e^(L_s - max); the weighted sum of the partial O rows then runs
@@ -488,9 +502,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
   const float L = mx + logf(den);
-  float acc[D / 32];
+  // Lane l owns columns [l * VW, (l + 1) * VW) of the row: one vector load
+  // per partial, eight partials in flight per step.
+  constexpr int VW = D / 32;
+  float acc[VW];
 #pragma unroll
-  for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
+  for (int i = 0; i < VW; ++i) acc[i] = 0.f;
   for (int base = 0; base < n_parts; base += 32) {
     // Lane i holds the weight and row of partial base + i (weight 0 past the
     // end, and for partials without a visible key, whose L is -inf).
@@ -502,25 +519,34 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
       wl = expf(part_l[rl] - L);
     }
     const int n = min(32, n_parts - base);
-    for (int i = 0; i < n; i += 4) {
-      float wv[4], x[4][D / 32];
+    for (int i = 0; i < n; i += 8) {
+      float wv[8], x[8][VW];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         wv[q] = __shfl_sync(0xffffffffu, wl, (i + q) & 31);
         const long long r = __shfl_sync(0xffffffffu, rl, (i + q) & 31);
-        const bool live = i + q < n && wv[q] != 0.f;
+        if (i + q < n && wv[q] != 0.f) {
+          load_vec(part_o + r * D + lane * VW, x[q]);
+        } else {
+          wv[q] = 0.f;
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k) x[q][k] = live ? part_o[r * D + k * 32 + lane] : 0.f;
-        if (!live) wv[q] = 0.f;
+          for (int k = 0; k < VW; ++k) x[q][k] = 0.f;
+        }
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int k = 0; k < D / 32; ++k) acc[k] = fmaf(wv[q], x[q][k], acc[k]);
+        for (int k = 0; k < VW; ++k) acc[k] = fmaf(wv[q], x[q][k], acc[k]);
     }
   }
+  uint32_t packed[VW / 2];
 #pragma unroll
-  for (int i = 0; i < D / 32; ++i) o[row * D + i * 32 + lane] = __float2bfloat16_rn(acc[i]);
+  for (int k = 0; k < VW / 2; ++k) packed[k] = pack_bf16x2(acc[2 * k], acc[2 * k + 1]);
+  if constexpr (VW == 4) {
+    *reinterpret_cast<uint2*>(o + row * D + lane * VW) = make_uint2(packed[0], packed[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(o + row * D + lane * VW) = packed[0];
+  }
   if (lane == 0) lse[row] = L;
 }
 
