@@ -6,6 +6,10 @@ causal, Q and K drawn with gain 2), inputs resident in HBM.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
     python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
 
+With --workload set to a decode workload (decode_*), a step is one decode
+call (Nq new queries per head against an Nk-key KV cache) and the metric is
+algorithmic bytes moved per second, bound by HBM.
+
 Prints one JSON line (rank 0). Multi-GPU runs are weak scaling: every rank
 runs its own batch of the same per-GPU size (attention over independent
 (batch, head) slices needs no exchange), timed on the device between
@@ -30,6 +34,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd/bwd TFLOP/s (bf16) and fraction of B200 dense BF16 peak"
+DECODE_METRIC = "decode attention: algorithmic HBM bytes per second (read q, K/V cache; write o, lse)"
 DEFAULT_WORKLOAD = "fwdbwd_b2_h16_n8192_d128_causal_peaky"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -183,8 +188,67 @@ def oracle_sample(w, seconds: float, max_slices: int = 64):
     return done, elapsed, n, threads
 
 
+def decode_oracle_sample(w, seconds: float, max_batches: int = 64):
+    """Times the fp64 decode oracle (as it stands) on whole batches of the
+    workload until about ``seconds`` have passed. Returns (algorithmic bytes
+    of the batches done, wall seconds, batches, threads)."""
+    import oracle
+    from exact_io_aware_56_b200 import make_decode_inputs, to_f64
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover - threadpoolctl missing
+        threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    bytes_batch = w.bytes_moved() / w.B
+    done, elapsed, n = 0.0, 0.0, 0
+    while n < max_batches and (elapsed < seconds or n == 0):
+        host = make_decode_inputs(1, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.seed + 7919 * (n + 1))
+        ref = {k: to_f64(v) for k, v in host.items()}
+        t0 = time.perf_counter()
+        oracle.attn_decode_ref(ref["q"], ref["k"], ref["v"], w.scale, w.causal)
+        elapsed += time.perf_counter() - t0
+        done += bytes_batch
+        n += 1
+    return done, elapsed, n, threads
+
+
+def decode_config(w, world):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+            "causal": w.causal, "global_batch": w.B * world,
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+
+def decode_reference_arm(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    times, threads = [], 1
+    for it in range(args.warmup + args.steps):
+        _, el, _, threads = decode_oracle_sample(w, 0.0, max_batches=1)
+        if it >= args.warmup:
+            times.append(el)
+    ms = 1e3 * sum(times) / len(times)
+    value = w.bytes_moved() / w.B / (ms * 1e-3) / 1e9
+    sample = f"one batch of {w.name} (fp64 decode oracle) per step"
+    line = {
+        "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(decode_config(w, 1), sample=sample),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def reference_arm(args):
-    from exact_io_aware_56_b200 import WORKLOADS
+    from exact_io_aware_56_b200 import DECODE_WORKLOADS, WORKLOADS
+
+    if args.workload in DECODE_WORKLOADS:
+        return decode_reference_arm(args, DECODE_WORKLOADS[args.workload])
 
     rank, world, _ = dist_env()
     if rank != 0:
@@ -372,10 +436,136 @@ def native_arm(args):
     return 0
 
 
+def decode_native_arm(args, w):
+    """One step = one fa_decode call on the resident cache; the decode
+    kernel's own time (split kernel, through the decode timing hook) gives
+    the roofline, the whole call (split + merge) the value."""
+    import torch
+
+    from exact_io_aware_56_b200 import fa, make_decode_inputs
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device; there is no CPU path")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl")
+    fa.lib()
+    host = make_decode_inputs(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.seed + rank)
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_decode(q, k, v, o, lse, w.causal, w.scale, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_check_device_error(stream) != fa.FA_OK:
+        raise RuntimeError("device watchdog fired during warm-up")
+    # Per-step events: [start, after the split kernel, end].
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for e in evs:  # torch creates the CUDA event on first record; the hook needs real handles
+        e[1].record(stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        t_start.record(stream)
+        for s in range(args.steps):
+            evs[s][0].record(stream)
+            fa.fa_profile_set_decode_event(evs[s][1])
+            step()
+            evs[s][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    fa.fa_profile_set_decode_event(None)
+    barrier(dev)
+    if fa.fa_check_device_error(stream) != fa.FA_OK:
+        raise RuntimeError("device watchdog fired during the timed steps")
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    value = w.bytes_moved() * args.steps * world / (ms_total * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    main_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    merge_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # The split kernel's algorithmic bytes: it reads q and the K/V cache
+    # (its partial results are working storage, not algorithmic traffic).
+    kv_q = 2 * w.B * w.Hkv * w.Nk * w.d * 2 + w.B * w.Hq * w.Nq * w.d * 2
+    achieved = kv_q / (main_ms * 1e-3) / 1e9
+    roofline = {
+        "bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        "frac": achieved / peak, "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+        "algorithmic_bytes_per_launch": kv_q,
+        "kernels": {"decode_kernel": {"ms": main_ms}, "decode_merge": {"ms": merge_ms}},
+    }
+    e2e = None
+    if args.e2e_steps > 0:
+        hin = {n: host[n].pin_memory() for n in host}
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse)]
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in (o, lse))
+        dins = {"q": q, "k": k, "v": v}
+
+        def e2e_step():
+            for n, t in dins.items():
+                t.copy_(hin[n], non_blocking=True)
+            step()
+            for src, dst in zip((o, lse), hout):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": w.bytes_moved() * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        done, secs, n, threads = decode_oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": done / secs / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} whole batches of {w.name}, fp64 decode oracle, {secs:.1f} s"}
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(decode_config(w, world),
+                       l2=f"K/V cache larger than L2 ({kv_q / 2**20:.0f} MiB per rank), no flush"),
+        "fraction_of_peak": value / world / peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return reference_arm(args)
+    from exact_io_aware_56_b200 import DECODE_WORKLOADS
+
+    if args.workload in DECODE_WORKLOADS:
+        return decode_native_arm(args, DECODE_WORKLOADS[args.workload])
     return native_arm(args)
 
 

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
-from exact_io_aware_56_b200 import WORKLOADS, Workload  # noqa: E402
+from exact_io_aware_56_b200 import DECODE_WORKLOADS, WORKLOADS, DecodeWorkload, Workload  # noqa: E402
 
 
 def _free_port():
@@ -63,6 +63,25 @@ def test_reference_arm_json(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["config"]["workload"] == "tiny_ref"
+
+
+def test_decode_reference_arm_json(monkeypatch, capsys):
+    tiny = DecodeWorkload("decode_tiny_ref", 2, 4, 2, 1, 300, 64, seed=5)
+    monkeypatch.setitem(DECODE_WORKLOADS, "decode_tiny_ref", tiny)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--impl", "reference", "--workload", "decode_tiny_ref", "--steps", "2", "--warmup", "1"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["metric"] == bench.DECODE_METRIC and line["config"]["Nk"] == 300
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_decode_workload_bytes():
+    w = DECODE_WORKLOADS["decode_b16_hq32_hkv8_nq1_nk8192_d128"]
+    kv = 2 * 16 * 8 * 8192 * 128 * 2
+    assert w.bytes_moved() == kv + 2 * 16 * 32 * 1 * 128 * 2 + 4 * 16 * 32
+    assert w.flops() == 4.0 * 16 * 32 * 1 * 8192 * 128
 
 
 def test_reference_arm_other_ranks_exit_quietly(monkeypatch, capsys):
