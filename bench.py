@@ -100,6 +100,34 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def captured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from the ncu table
+    in profiles/traffic.md, or None when there is no row or the kernel's
+    sources changed since the capture (sha256 of their concatenation)."""
+    import hashlib
+
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.md")) as f:
+            lines = f.read().splitlines()
+    except OSError:
+        return None
+    for ln in lines:
+        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
+        if len(cells) != 5 or cells[0] != kernel or cells[1] != workload:
+            continue
+        m = hashlib.sha256()
+        try:
+            for src in cells[2].split():
+                with open(os.path.join(ROOT, "exact_io_aware_56_b200", "csrc", src), "rb") as f:
+                    m.update(f.read())
+        except OSError:
+            return None
+        if m.hexdigest()[:16] != cells[3]:
+            return None
+        return int(cells[4])
+    return None
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -366,7 +394,9 @@ def native_arm(args):
     dom = max((kn for kn in ("fwd", "bwd_main") if kn in kernels), key=lambda kn: kernels[kn]["ms"])
     roofline = {
         "bound": "tensor", "kernel": dom, "achieved": kernels[dom]["tflops"], "peak": peak, "unit": "TFLOP/s",
-        "frac": kernels[dom]["frac"], "traffic": None,
+        "frac": kernels[dom]["frac"], "traffic": captured_traffic(dom, w.name),
+        "traffic_algorithmic": "fwd: q, k, v read, o (+ o_resid), lse written; "
+                               "bwd: q, k, v, dO, L, D read, dk, dv written, dQ fp32 accumulator",
         "peak_source": f"{peak_src} bf16 dense (burst)",
         "kernels": {kn: {x: kernels[kn][x] for x in ("ms", "tflops", "frac") if x in kernels[kn]}
                     for kn in kernels},
@@ -500,7 +530,8 @@ def decode_native_arm(args, w):
     achieved = kv_q / (main_ms * 1e-3) / 1e9
     roofline = {
         "bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": peak, "unit": "GB/s",
-        "frac": achieved / peak, "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+        "frac": achieved / peak, "traffic": captured_traffic("decode_kernel", w.name),
+        "peak_source": f"{peak_src} copy bandwidth",
         "algorithmic_bytes_per_launch": kv_q,
         "kernels": {"decode_kernel": {"ms": main_ms}, "decode_merge": {"ms": merge_ms}},
     }

@@ -96,3 +96,21 @@ def test_workload_flops():
     assert w.fwd_flops() == pytest.approx(549.755813888e9)
     assert w.bwd_flops() == pytest.approx(2.5 * 549.755813888e9)
     assert WORKLOADS["fwd_b1_h1_n128_d64"].fwd_flops() == 4 * 128 * 128 * 64
+
+
+def test_captured_traffic_requires_unchanged_sources(tmp_path, monkeypatch):
+    import hashlib
+
+    csrc = tmp_path / "exact_io_aware_56_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_bytes(b"kernel source v1")
+    digest = hashlib.sha256(b"kernel source v1").hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.md").write_text(
+        "| kernel | workload | sources | sha256/16 | traffic bytes |\n|---|---|---|---|---|\n"
+        f"| kern | wl | k.cu | {digest} | 12345 |\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.captured_traffic("kern", "wl") == 12345
+    assert bench.captured_traffic("kern", "other") is None
+    (csrc / "k.cu").write_bytes(b"kernel source v2")
+    assert bench.captured_traffic("kern", "wl") is None
