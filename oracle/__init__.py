@@ -34,6 +34,13 @@ from .attention import (  # noqa: F401
     visible,
     kv_head_of,
 )
+from .fp8 import (  # noqa: F401
+    attn_fwd_fp8_ref,
+    dequantize_blocks,
+    e4m3_decode,
+    e4m3_encode,
+    quantize_blocks,
+)
 from .memory import (  # noqa: F401
     naive_score_bytes,
     flash_state_bytes,
