@@ -58,8 +58,9 @@ def _positive_grid():
 
 def e4m3_encode(x) -> np.ndarray:
     """Nearest e4m3 code of each float (ties to the even code, i.e. the one
-    whose mantissa's last bit is 0), saturating at +-448. NaN is not
-    accepted."""
+    whose mantissa's last bit is 0), saturating at +-448. The sign bit is
+    the sign of x, zeros included, as in IEEE format conversions (a negative
+    value that rounds to zero gives 0x80). NaN is not accepted."""
     x = np.asarray(x, dtype=np.float64)
     if np.isnan(x).any():
         raise ValueError("NaN has no rounding target")
@@ -71,9 +72,7 @@ def e4m3_encode(x) -> np.ndarray:
     pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((codes[hi] & 1) == 0))
     idx = np.where(pick_hi, hi, lo)
     out = codes[idx].astype(np.uint8)
-    # Negative values carry the sign bit; -0 and +0 both encode as 0x00.
-    neg = (x < 0) & (out != 0)
-    return np.where(neg, out | 0x80, out).astype(np.uint8)
+    return np.where(np.signbit(x), out | 0x80, out).astype(np.uint8)
 
 
 def quantize_blocks(x, block_rows: int | None = BLOCK_ROWS):
