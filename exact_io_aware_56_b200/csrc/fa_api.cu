@@ -256,6 +256,44 @@ int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, co
                   workspace_bytes, stream, window, prefix);
 }
 
+int fa_quantize_fp8(const void* x, void* codes, float* scales, int BH, int N, int d, int per_head, void* stream) {
+  if (!x || !codes || !scales) return FA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FA_ERR_INVALID_ARGUMENT;
+  if (BH <= 0 || N <= 0 || (per_head != 0 && per_head != 1)) return FA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(BH) * N * d >= (1LL << 40)) return FA_ERR_UNSUPPORTED;
+  DevState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != FA_OK) return rc;
+  cudaError_t e = launch_quantize_fp8(x, codes, scales, BH, N, d, per_head, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
+int fa_fwd_fp8(const void* q8, const float* sq, const void* k8, const float* sk, const void* v8, const float* sv,
+               void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  if (!q8 || !sq || !k8 || !sk || !v8 || !sv || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
+  const void* ptrs[] = {q8, k8, v8, o, lse};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_INVALID_ARGUMENT;
+  const void* sptrs[] = {sq, sk, sv};
+  for (const void* p : sptrs)
+    if (reinterpret_cast<uintptr_t>(p) & 3u) return FA_ERR_INVALID_ARGUMENT;
+  int rc = check_shape(B, Hq, Hkv, N, d, causal, scale);
+  if (rc != FA_OK) return rc;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  DevState* st = nullptr;
+  if ((rc = device_state(&st)) != FA_OK) return rc;
+  // e4m3 tensors: 128 one-byte columns per row, boxes of 128 columns x 128 rows.
+  CUtensorMap tq, tk, tv;
+  if (!encode_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q8, d, N, B * Hq, 128, 128) ||
+      !encode_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k8, d, N, B * Hkv, 128, 128) ||
+      !encode_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v8, d, N, B * Hkv, 128, 128))
+    return FA_ERR_UNSUPPORTED;
+  AttnShape s{B, Hq, Hkv, N, d, causal, scale};
+  cudaError_t e = launch_fwd_fp8(s, tq, tk, tv, o, lse, sq, sk, sv, make_ctl(st), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   if (check_decode_shape(B, Hq, Hkv, Nq, Nk, d, 0, 1.f) != FA_OK) return 0;
   DecodeShape s{B, Hq, Hkv, Nq, Nk, d, 0, 1.f};

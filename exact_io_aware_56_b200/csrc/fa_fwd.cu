@@ -63,11 +63,15 @@ constexpr float kRescaleThreshold = 0.0f;  // log2 units
 // so the extra FMA-pipe instructions only add issue slots.
 constexpr int kPolyPer32 = 0;
 
-template <int D>
+// F8: e4m3 Q, K, V with block scales (the FP8 mode); otherwise bf16.
+template <int D, bool F8 = false>
 struct FwdCfg {
-  static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kBoxBytes = kBN * 64 * 2;       // one 64-column TMA box of a 128-row tile
-  static constexpr int kBoxes = D / 64;
+  static constexpr int kElem = F8 ? 1 : 2;              // bytes per element
+  static constexpr int kBoxCols = 128 / kElem;          // elements per 128-byte swizzle row
+  static constexpr int kKStep = 32 / kElem;             // MMA K per instruction (16 bf16, 32 e4m3)
+  static constexpr int kStages = (D * kElem == 256) ? 2 : 4;
+  static constexpr int kBoxBytes = kBN * 128;           // one 128-byte-wide TMA box of a 128-row tile
+  static constexpr int kBoxes = D * kElem / 128;
   static constexpr int kTileBytes = kBoxBytes * kBoxes;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = 2 * kTileBytes;
@@ -80,6 +84,14 @@ struct FwdCfg {
   static_assert(kSmemBytes > 114 * 1024, "one CTA per SM (owns all tensor memory)");
 };
 
+// Block scales of the FP8 mode: Q and K per 128-row block of a head
+// ([B*Hq][nb], [B*Hkv][nb]), V per head ([B*Hkv]).
+struct Fp8Scales {
+  const float* sq;
+  const float* sk;
+  const float* sv;
+};
+
 struct FwdArgs {
   __nv_bfloat16* o;
   __nv_bfloat16* o_resid;  // optional: bf16(O - bf16(O)), the rounding residual of o
@@ -89,6 +101,7 @@ struct FwdArgs {
   int window;  // left window (a huge value when there is none), mask kind 2
   int prefix;  // prefix length, mask kind 2
   float scale_log2;
+  Fp8Scales f8;
   LaunchCtl ctl;
 };
 
@@ -108,11 +121,13 @@ __device__ __forceinline__ bool visible2(int i, int j, int window, int prefix) {
 }
 
 // MASK: 0 none, 1 causal, 2 causal with a left window and/or a prefix.
-template <int D, int MASK>
+// F8: e4m3 operands with block scales (FP8 mode, masks 0 and 1).
+template <int D, int MASK, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
+  static_assert(!F8 || MASK != 2, "FP8 mode covers the unmasked and causal forward");
   constexpr int ST = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -200,8 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(&tmQ, &bars->q_full, smem + C::kOffQ + t * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                      q0 + t * kBM, bh);
+          tma_load_3d(&tmQ, &bars->q_full, smem + C::kOffQ + t * C::kTileBytes + x * C::kBoxBytes,
+                      x * C::kBoxCols, q0 + t * kBM, bh);
       const int n = n_t[1];
       for (int j = 0; j < n; ++j) {
         const int s = j % ST;
@@ -211,15 +226,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
 #pragma unroll
           for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                        key_tile(j) * kBN, kvh);
+            tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes,
+                        x * C::kBoxCols, key_tile(j) * kBN, kvh);
           k_last[s] = u;
         }
         mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
 #pragma unroll
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes, x * 64,
-                      key_tile(j) * kBN, kvh);
+          tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes,
+                      x * C::kBoxCols, key_tile(j) * kBN, kvh);
         v_last[s] = u;
       }
       // Every copy issued must land before the CTA may exit.
@@ -233,26 +248,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, false, true);
+      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(kBM, kBN, false, false) : idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(kBM, D, false, true) : idesc_bf16(kBM, D, false, true);
+      constexpr int KS = C::kKStep;
       const uint32_t tS[2] = {tmem, tmem + 128u};
       const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
       auto issue_s = [&](int t, int j) {
         const uint32_t qa = sQ + t * C::kTileBytes;
         const uint32_t ka = sK + (j % ST) * C::kTileBytes;
+        // Each K step is 32 bytes of a 128-byte swizzle row (16 bf16 or 32 e4m3).
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
+        for (int k = 0; k < D / KS; ++k) {
           const uint32_t off = (k / 4) * C::kBoxBytes + (k % 4) * 32;
-          mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
+          if constexpr (F8)
+            mma_ss_f8(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
+          else
+            mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
         }
         mma_commit(&bars->s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t va = sV + (j % ST) * C::kTileBytes;
+        // P: KS keys per step = 8 tensor-memory columns (bf16 pairs or e4m3
+        // quads); V: KS key rows of 128 bytes (MN-major).
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k)
-          mma_ts(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * 2048, C::kBoxBytes, 1024), idesc_pv,
-                 (j > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < kBN / KS; ++k) {
+          if constexpr (F8)
+            mma_ts_f8(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * KS * 128, C::kBoxBytes, 1024), idesc_pv,
+                      (j > 0 || k > 0) ? 1u : 0u);
+          else
+            mma_ts(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * KS * 128, C::kBoxBytes, 1024), idesc_pv,
+                   (j > 0 || k > 0) ? 1u : 0u);
+        }
       };
       const int n0 = n_t[0], n1 = n_t[1];
       bool ok = wait_bar(&bars->q_full, 0, w) && wait_bar(&bars->k_full[0], 0, w);
@@ -299,7 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + t * 128u;
     const uint32_t tO = tmem + lane_off + 256u + t * D;
     const int n = n_t[t];
-    const float sl2 = a.scale_log2;
+    // FP8 mode: the scores come out of the MMA in units of sq * sk (the Q
+    // tile's and the K tile's block scales); both fold into the exponent's
+    // scale, per tile.
+    // (The second tile of the last pair may start past N; its rows are never
+    // written, and its block index is clamped into the scale array.)
+    const float sl2_q =
+        F8 ? a.scale_log2 * a.f8.sq[static_cast<size_t>(bh) * a.nk + min((q0 + t * kBM) / kBM, a.nk - 1)]
+           : a.scale_log2;
     const int lim = MASK == 1 ? min(row, a.N - 1) : a.N - 1;  // last visible key (kinds 0, 1)
     const int qt0 = q0 + t * kBM;                               // first query of this tile
     float m = -CUDART_INF_F;  // running max of scale*log2(e)*s
@@ -311,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[kBN];
       tmem_ld128(tS, sr);
+      const float sl2 = F8 ? sl2_q * a.f8.sk[static_cast<size_t>(kvh) * a.nk + key_tile(j)] : sl2_q;
       if (MASK != 2) {
         if (j == n - 1) {
           const int k0 = j * kBN;
@@ -360,24 +395,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // A row with no visible key so far has m = -inf: its masked scores
       // must give exp(-inf) = 0, not exp(-inf + inf).
-      const float neg_m = (MASK == 2 && m == -CUDART_INF_F) ? 0.f : -m;
+      // FP8 mode writes P as e4m3 of 2^8 p (headroom below 1 against
+      // underflow, exact to undo): the +8 rides on the exponent.
+      const float neg_m = ((MASK == 2 && m == -CUDART_INF_F) ? 0.f : -m) + (F8 ? 8.f : 0.f);
       float ps[8];  // 8 independent partial row sums
 #pragma unroll
       for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+      if constexpr (F8) {
+        // 64 scores -> 16 columns of four e4m3 each.
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < kBN / 64; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float x0 = fmaf(__uint_as_float(sr[c * 32 + 2 * i]), sl2, neg_m);
-          const float x1 = fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, neg_m);
-          const float p0 = (2 * i < kPolyPer32) ? exp2_poly(x0) : ex2(x0);
-          const float p1 = (2 * i + 1 < kPolyPer32) ? exp2_poly(x1) : ex2(x1);
-          ps[(2 * i) & 7] += p0;
-          ps[(2 * i + 1) & 7] += p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            float p4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              p4[e] = ex2(fmaf(__uint_as_float(sr[c * 64 + 4 * i + e]), sl2, neg_m));
+              ps[(4 * i + e) & 7] += p4[e];
+            }
+            pk[i] = pack_e4m3x4(p4[0], p4[1], p4[2], p4[3]);
+          }
+          tmem_st16(tS + c * 16, pk);
         }
-        tmem_st16(tS + c * 16, pk);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(__uint_as_float(sr[c * 32 + 2 * i]), sl2, neg_m);
+            const float x1 = fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, neg_m);
+            const float p0 = (2 * i < kPolyPer32) ? exp2_poly(x0) : ex2(x0);
+            const float p1 = (2 * i + 1 < kPolyPer32) ? exp2_poly(x1) : ex2(x1);
+            ps[(2 * i) & 7] += p0;
+            ps[(2 * i + 1) & 7] += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
       }
       const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       if (rescale) {
@@ -412,7 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->o_final[t], 0, w));
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      // FP8 mode: l sums 2^8 p, O sums (2^8 p) V_codes; V's head scale turns
+      // codes into values.
+      const float inv_l = F8 ? a.f8.sv[kvh] / l : 1.f / l;
       __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.N + row) * D;
       __nv_bfloat16* rrow = a.o_resid ? a.o_resid + (static_cast<size_t>(bh) * a.N + row) * D : nullptr;
 #pragma unroll
@@ -441,7 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (row < a.N) a.lse[static_cast<size_t>(bh) * a.N + row] = (m + lg2(l)) * 0.69314718055994530942f;
+      if (row < a.N)
+        a.lse[static_cast<size_t>(bh) * a.N + row] = (m + lg2(l) - (F8 ? 8.f : 0.f)) * 0.69314718055994530942f;
     }
   }
 
@@ -454,11 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int MASK>
+template <int D, int MASK, bool F8 = false>
 cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
-  using C = FwdCfg<D>;
-  auto kern = fwd_kernel<D, MASK>;
+                         void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream,
+                         Fp8Scales f8 = Fp8Scales{nullptr, nullptr, nullptr}) {
+  using C = FwdCfg<D, F8>;
+  auto kern = fwd_kernel<D, MASK, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
@@ -473,10 +533,12 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.n_pairs = (s.N + 2 * kBM - 1) / (2 * kBM);
   // Causal units differ in length: keep strict longest-first order over all
   // heads. Non-causal units are equal: group heads for L2 locality.
-  a.group = MASK == 1 ? a.BH : l2_head_group(static_cast<long long>(4) * s.N * D / (s.Hq / s.Hkv), a.BH);
+  a.group = MASK == 1 ? a.BH
+                      : l2_head_group(static_cast<long long>(2 * C::kElem) * s.N * D / (s.Hq / s.Hkv), a.BH);
   a.window = s.window < 0 ? 0x3fffffff : s.window;
   a.prefix = s.prefix;
   a.scale_log2 = s.scale * 1.4426950408889634f;
+  a.f8 = f8;
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.n_pairs) * a.BH;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -498,6 +560,15 @@ cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensor
     default: return launch_fwd_t<128, 2>(FA_FWD_ARGS);
   }
 #undef FA_FWD_ARGS
+}
+
+cudaError_t launch_fwd_fp8(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           void* o, float* lse, const float* sq, const float* sk, const float* sv,
+                           const LaunchCtl& ctl, cudaStream_t stream) {
+  if (s.d != 128 || s.mask_kind() == 2) return cudaErrorInvalidValue;
+  const Fp8Scales f8{sq, sk, sv};
+  if (s.causal) return launch_fwd_t<128, 1, true>(s, tq, tk, tv, o, nullptr, lse, ctl, stream, f8);
+  return launch_fwd_t<128, 0, true>(s, tq, tk, tv, o, nullptr, lse, ctl, stream, f8);
 }
 
 }  // namespace fa

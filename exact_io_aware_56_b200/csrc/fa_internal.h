@@ -51,6 +51,17 @@ bool encode_f32_tile_map(CUtensorMap* map, const void* base, int cols, int rows,
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream);
 
+// FP8 mode (d = 128, masks 0 and 1): q, k, v are e4m3 codes behind 1-byte
+// tensor maps with 128-column boxes; sq, sk, sv the block scales.
+cudaError_t launch_fwd_fp8(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           void* o, float* lse, const float* sq, const float* sk, const float* sv,
+                           const LaunchCtl& ctl, cudaStream_t stream);
+
+// e4m3 block quantization of a bf16 tensor [BH][N][d]: scales per 128-row
+// block ([BH][ceil(N/128)]) or per head ([BH]); see fa.h.
+cudaError_t launch_quantize_fp8(const void* x, void* codes, float* scales, int BH, int N, int d, int per_head,
+                                cudaStream_t stream);
+
 size_t bwd_workspace_bytes(const AttnShape& s);
 
 cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

@@ -54,6 +54,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_masked.restype = i
     L.fa_bwd_masked.argtypes = [vp] * 10 + [i, i, i, i, i, i, i, f, vp, sz, vp]
     L.fa_bwd_masked.restype = i
+    L.fa_quantize_fp8.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    L.fa_quantize_fp8.restype = i
+    L.fa_fwd_fp8.argtypes = [vp] * 8 + [i, i, i, i, i, i, f, vp]
+    L.fa_fwd_fp8.restype = i
     L.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
     L.fa_decode_workspace_bytes.restype = sz
     L.fa_decode.argtypes = [vp] * 5 + [i, i, i, i, i, i, i, f, vp, sz, vp]
@@ -176,6 +180,38 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, worksp
         raise FaError(rc, name)
 
 
+def fa_quantize_fp8(x, codes, scales, per_head: bool, stream=None) -> None:
+    """e4m3 block quantization of ``x`` [B, H, N, d] bf16 into ``codes``
+    (uint8, like x) and ``scales`` (fp32: [B*H, ceil(N/128)] per 128-row
+    block, or [B*H] per head)."""
+    if x.dim() != 4:
+        raise ValueError("x must be [B, H, N, d]")
+    B, H, N, d = x.shape
+    nb = (N + 127) // 128
+    xa = _check_tensor("x", x, torch.bfloat16, (B, H, N, d))
+    ca = _check_tensor("codes", codes, torch.uint8, (B, H, N, d))
+    sa = _check_tensor("scales", scales, torch.float32, (B * H,) if per_head else (B * H, nb))
+    rc = lib().fa_quantize_fp8(xa, ca, sa, B * H, N, d, int(bool(per_head)), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_quantize_fp8")
+
+
+def fa_fwd_fp8(q8, sq, k8, sk, v8, sv, o, lse, causal: bool, scale: float, stream=None) -> None:
+    """FP8-mode forward (d = 128): e4m3 codes ``q8`` [B,Hq,N,d], ``k8``/``v8``
+    [B,Hkv,N,d] (uint8) with block scales ``sq`` [B*Hq, nb], ``sk``
+    [B*Hkv, nb], ``sv`` [B*Hkv]; writes ``o`` (bf16) and ``lse`` (fp32)."""
+    B, Hq, Hkv, N, d = _shapes(q8, k8)
+    nb = (N + 127) // 128
+    u8, f32 = torch.uint8, torch.float32
+    args = [_check_tensor("q8", q8, u8, (B, Hq, N, d)), _check_tensor("sq", sq, f32, (B * Hq, nb)),
+            _check_tensor("k8", k8, u8, (B, Hkv, N, d)), _check_tensor("sk", sk, f32, (B * Hkv, nb)),
+            _check_tensor("v8", v8, u8, (B, Hkv, N, d)), _check_tensor("sv", sv, f32, (B * Hkv,)),
+            _check_tensor("o", o, torch.bfloat16, (B, Hq, N, d)), _check_tensor("lse", lse, f32, (B, Hq, N))]
+    rc = lib().fa_fwd_fp8(*args, B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_fp8")
+
+
 def fa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int) -> int:
     return int(lib().fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d))
 
@@ -271,3 +307,27 @@ def attention_decode(q, k, v, causal: bool = True, scale: float | None = None, w
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     fa_decode(q, k, v, o, lse, causal, scale, workspace, stream)
     return o, lse
+
+
+def quantize_fp8(x, per_head: bool = False, stream=None):
+    """Allocates and returns ``(codes, scales)`` for :func:`fa_quantize_fp8`."""
+    B, H, N, d = x.shape
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    shape = (B * H,) if per_head else (B * H, (N + 127) // 128)
+    scales = torch.empty(shape, dtype=torch.float32, device=x.device)
+    fa_quantize_fp8(x, codes, scales, per_head, stream)
+    return codes, scales
+
+
+def attention_forward_fp8(q, k, v, causal: bool, scale: float | None = None, stream=None):
+    """Quantizes bf16 ``q``, ``k`` (per 128-row block) and ``v`` (per head) and
+    runs :func:`fa_fwd_fp8`. Returns ``(o, lse, (q8, sq, k8, sk, v8, sv))``."""
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    scale = d ** -0.5 if scale is None else scale
+    q8, sq = quantize_fp8(q, False, stream)
+    k8, sk = quantize_fp8(k, False, stream)
+    v8, sv = quantize_fp8(v, True, stream)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    fa_fwd_fp8(q8, sq, k8, sk, v8, sv, o, lse, causal, scale, stream)
+    return o, lse, (q8, sq, k8, sk, v8, sv)

@@ -177,6 +177,43 @@ int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, co
                   int prefix, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * FP8 mode (e4m3 with block scaling).
+ *
+ * "FlashAttention: IO-aware exact attention" ("The generations") lists FP8
+ * support with block scaling for FlashAttention-3, and ("The honest limits")
+ * notes that FP8 changes rounding. Here: e4m3 codes (1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, no infinities, largest finite 448) with one
+ * fp32 scale per block; a value is code * scale.
+ *
+ * fa_quantize_fp8 quantizes a bf16 tensor x [BH][N][d] (d = 64 or 128) into
+ * codes (uint8, same layout) and scales:
+ *   per_head = 0: one scale per 128-row block, scales [BH][ceil(N/128)];
+ *   per_head = 1: one scale per head,          scales [BH].
+ * scale = amax / 448 (amax = largest |x| of the block; 1 for an all-zero
+ * block), codes = e4m3(x * (448 / amax)) rounded to nearest even and
+ * saturated, both fp32 operations correctly rounded. Q and K use 128-row
+ * blocks, V one scale per head. Three small kernels on `stream`.
+ *
+ * fa_fwd_fp8 is the forward of fa_fwd on the dequantized tensors
+ * (q_hat = q8 * sq of its 128-row block, k_hat likewise, v_hat = v8 * sv
+ * of its head), for d = 128: q8 [B][Hq][N][128], k8 and v8 [B][Hkv][N][128]
+ * e4m3 codes (16-byte aligned); sq [B*Hq][ceil(N/128)], sk [B*Hkv][ceil(N/128)],
+ * sv [B*Hkv] fp32 (4-byte aligned); o bf16 [B][Hq][N][128], lse fp32
+ * [B][Hq][N]. Both products run on e4m3 operands with fp32 accumulation;
+ * the softmax weights enter the second one as e4m3 of 2^8 p, the main
+ * rounding beyond the inputs' own.
+ *
+ * Returns FA_OK; FA_ERR_INVALID_ARGUMENT (null or misaligned pointer,
+ * non-positive size, bad causal or per_head flag, non-finite or
+ * non-positive scale); FA_ERR_UNSUPPORTED (d other than 128 for the
+ * forward, 64/128 for quantization; Hq not a multiple of Hkv; size limits;
+ * device not compute capability 10.0); FA_ERR_CUDA on a launch failure.
+ */
+int fa_quantize_fp8(const void* x, void* codes, float* scales, int BH, int N, int d, int per_head, void* stream);
+int fa_fwd_fp8(const void* q8, const float* sq, const void* k8, const float* sk, const void* v8, const float* sv,
+               void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/*
  * Decode / short-query attention against a KV cache.
  *
  * Nq new queries per head attend to an Nk-key cache, 1 <= Nq <= Nk. The
