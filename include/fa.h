@@ -200,8 +200,10 @@ int fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, co
  * e4m3 codes (16-byte aligned); sq [B*Hq][ceil(N/128)], sk [B*Hkv][ceil(N/128)],
  * sv [B*Hkv] fp32 (4-byte aligned); o bf16 [B][Hq][N][128], lse fp32
  * [B][Hq][N]. Both products run on e4m3 operands with fp32 accumulation;
- * the softmax weights enter the second one as e4m3 of 2^8 p, the main
- * rounding beyond the inputs' own.
+ * the softmax weights enter the second one as e4m3 of 2^(x + 4), x the
+ * exponent against a running row max that may lag the true one by up to 4
+ * (the rescale of O is skipped for smaller growth), the main rounding
+ * beyond the inputs' own.
  *
  * Returns FA_OK; FA_ERR_INVALID_ARGUMENT (null or misaligned pointer,
  * non-positive size, bad causal or per_head flag, non-finite or
