@@ -6,6 +6,11 @@ causal, Q and K drawn with gain 2), inputs resident in HBM.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
     python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...
 
+With --workload set to an FP8 workload (fwd_fp8_*), a step is one FP8-mode
+forward on inputs quantized to e4m3 beforehand (quantization is in the e2e
+leg, not in the kernel timing), against twice the measured bf16 peak (the
+nominal FP8 : bf16 ratio of the tensor cores).
+
 With --workload set to a decode workload (decode_*), a step is one decode
 call (Nq new queries per head against an Nk-key KV cache) and the metric is
 algorithmic bytes moved per second, bound by HBM.
@@ -34,6 +39,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd/bwd TFLOP/s (bf16) and fraction of B200 dense BF16 peak"
+FP8_METRIC = "attention forward TFLOP/s in FP8 mode (e4m3 operands, block scales) and fraction of B200 dense FP8 peak"
 DECODE_METRIC = "decode attention: algorithmic HBM bytes per second (read q, K/V cache; write o, lse)"
 DEFAULT_WORKLOAD = "fwdbwd_b2_h16_n8192_d128_causal_peaky"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -272,11 +278,67 @@ def decode_reference_arm(args, w):
     return 0
 
 
+def fp8_oracle_sample(w, seconds: float, max_slices: int = 64):
+    """Times the fp64 FP8-mode oracle (quantize with the oracle, then attention
+    on the dequantized tensors) on whole (batch, head) slices. Returns
+    (algorithmic FLOPs done, wall seconds, slices, threads)."""
+    import oracle
+    from exact_io_aware_56_b200 import make_inputs, to_f64
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover - threadpoolctl missing
+        threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    flops_slice = w.fwd_flops() / (w.B * w.Hq)
+    done, elapsed, n = 0.0, 0.0, 0
+    while n < max_slices and (elapsed < seconds or n == 0):
+        host = make_inputs(1, 1, 1, w.N, w.d, w.seed + 7919 * (n + 1), w.qk_gain, False)
+        ref = {k: to_f64(v) for k, v in host.items()}
+        t0 = time.perf_counter()
+        q8, sq = oracle.quantize_blocks(ref["q"])
+        k8, sk = oracle.quantize_blocks(ref["k"])
+        v8, sv = oracle.quantize_blocks(ref["v"], None)
+        oracle.attn_fwd_fp8_ref(q8, sq, k8, sk, v8, sv, w.causal, w.scale)
+        elapsed += time.perf_counter() - t0
+        done += flops_slice
+        n += 1
+    return done, elapsed, n, threads
+
+
+def fp8_reference_arm(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    times, threads = [], 1
+    for it in range(args.warmup + args.steps):
+        _, el, _, threads = fp8_oracle_sample(w, 0.0, max_slices=1)
+        if it >= args.warmup:
+            times.append(el)
+    ms = 1e3 * sum(times) / len(times)
+    value = w.fwd_flops() / (w.B * w.Hq) / (ms * 1e-3) / 1e12
+    sample = f"one (batch, head) slice of {w.name} (fp64 FP8-mode oracle: quantize + attention) per step"
+    line = {
+        "impl": "reference", "metric": FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def reference_arm(args):
-    from exact_io_aware_56_b200 import DECODE_WORKLOADS, WORKLOADS
+    from exact_io_aware_56_b200 import DECODE_WORKLOADS, FP8_WORKLOADS, WORKLOADS
 
     if args.workload in DECODE_WORKLOADS:
         return decode_reference_arm(args, DECODE_WORKLOADS[args.workload])
+    if args.workload in FP8_WORKLOADS:
+        return fp8_reference_arm(args, FP8_WORKLOADS[args.workload])
 
     rank, world, _ = dist_env()
     if rank != 0:
@@ -466,6 +528,119 @@ def native_arm(args):
     return 0
 
 
+def fp8_native_arm(args, w):
+    """One step = one fa_fwd_fp8 call on e4m3 codes and scales resident in
+    HBM (quantized once by fa_quantize_fp8 before the timed region)."""
+    import torch
+
+    from exact_io_aware_56_b200 import fa, make_inputs
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device; there is no CPU path")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl")
+    fa.lib()
+    host = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + rank, w.qk_gain, False)
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    stream = torch.cuda.current_stream(dev)
+    q8, sq = fa.quantize_fp8(q, False, stream)
+    k8, sk = fa.quantize_fp8(k, False, stream)
+    v8, sv = fa.quantize_fp8(v, True, stream)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+
+    def step():
+        fa.fa_fwd_fp8(q8, sq, k8, sk, v8, sv, o, lse, w.causal, w.scale, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_check_device_error(stream) != fa.FA_OK:
+        raise RuntimeError("device watchdog fired during warm-up")
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.3)
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dev)
+    if fa.fa_check_device_error(stream) != fa.FA_OK:
+        raise RuntimeError("device watchdog fired during the timed steps")
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    value = w.fwd_flops() * args.steps * world / (ms_total * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = w.fwd_flops() / (ms_total / args.steps * 1e-3) / 1e12
+    roofline = {
+        "bound": "tensor", "kernel": "fwd_fp8", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": achieved / peak, "traffic": captured_traffic("fwd_fp8", w.name),
+        "peak_source": f"{peak_src} bf16 dense (burst) x 2, the nominal FP8 : bf16 ratio",
+    }
+    e2e = None
+    if args.e2e_steps > 0:
+        hin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse)]
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in (o, lse))
+
+        def e2e_step():
+            for n, t in (("q", q), ("k", k), ("v", v)):
+                t.copy_(hin[n], non_blocking=True)
+            fa.fa_quantize_fp8(q, q8, sq, False, stream)
+            fa.fa_quantize_fp8(k, k8, sk, False, stream)
+            fa.fa_quantize_fp8(v, v8, sv, True, stream)
+            step()
+            for src, dst in zip((o, lse), hout):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": w.fwd_flops() * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops, secs, n, threads = fp8_oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} whole (batch, head) slices of {w.name}, fp64 FP8-mode oracle, {secs:.1f} s"}
+    in_bytes = sum(t.numel() for t in (q8, k8, v8))
+    line = {
+        "metric": FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "qk_gain": w.qk_gain, "global_batch": w.B * world,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"e4m3 inputs {in_bytes / 2**20:.0f} MiB per rank, compute-bound, no flush"},
+        "fraction_of_peak": value / world / peak,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def decode_native_arm(args, w):
     """One step = one fa_decode call on the resident cache; the decode
     kernel's own time (split kernel, through the decode timing hook) gives
@@ -593,10 +768,12 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return reference_arm(args)
-    from exact_io_aware_56_b200 import DECODE_WORKLOADS
+    from exact_io_aware_56_b200 import DECODE_WORKLOADS, FP8_WORKLOADS
 
     if args.workload in DECODE_WORKLOADS:
         return decode_native_arm(args, DECODE_WORKLOADS[args.workload])
+    if args.workload in FP8_WORKLOADS:
+        return fp8_native_arm(args, FP8_WORKLOADS[args.workload])
     return native_arm(args)
 
 

@@ -8,6 +8,7 @@ is missing or no CUDA device is present, and there is no CPU fallback.
 
 from .inputs import (  # noqa: F401
     DECODE_WORKLOADS,
+    FP8_WORKLOADS,
     WORKLOADS,
     DecodeWorkload,
     Workload,
@@ -18,5 +19,5 @@ from .inputs import (  # noqa: F401
     workload_inputs,
 )
 
-__all__ = ["DECODE_WORKLOADS", "WORKLOADS", "DecodeWorkload", "Workload", "make_decode_inputs", "make_inputs",
+__all__ = ["DECODE_WORKLOADS", "FP8_WORKLOADS", "WORKLOADS", "DecodeWorkload", "Workload", "make_decode_inputs", "make_inputs",
            "sample_rows", "to_f64", "workload_inputs"]

@@ -67,6 +67,17 @@ WORKLOADS = {
 }
 
 
+# FP8-mode forward workloads: the same shapes and input recipe as the bf16
+# workloads above, quantized to e4m3 (Q, K per 128-row block, V per head)
+# before the timed forward.
+FP8_WORKLOADS = {
+    "fwd_fp8_b2_h16_n8192_d128_causal_peaky": Workload("fwd_fp8_b2_h16_n8192_d128_causal_peaky", 2, 16, 16, 8192,
+                                                       128, True, False, qk_gain=2.0, seed=1002),
+    "fwd_fp8_gqa_b1_hq32_hkv8_n16384_d128_causal": Workload("fwd_fp8_gqa_b1_hq32_hkv8_n16384_d128_causal", 1, 32,
+                                                            8, 16384, 128, True, False, seed=1003),
+}
+
+
 @dataclass(frozen=True)
 class DecodeWorkload:
     """Decode against a KV cache: Nq new queries per head, an Nk-key cache.

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
-from exact_io_aware_56_b200 import DECODE_WORKLOADS, WORKLOADS, DecodeWorkload, Workload  # noqa: E402
+from exact_io_aware_56_b200 import DECODE_WORKLOADS, FP8_WORKLOADS, WORKLOADS, DecodeWorkload, Workload  # noqa: E402
 
 
 def _free_port():
@@ -75,6 +75,16 @@ def test_decode_reference_arm_json(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["metric"] == bench.DECODE_METRIC and line["config"]["Nk"] == 300
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_fp8_reference_arm_json(monkeypatch, capsys):
+    tiny = Workload("fwd_fp8_tiny", 1, 2, 1, 256, 128, True, False, seed=4)
+    monkeypatch.setitem(FP8_WORKLOADS, "fwd_fp8_tiny", tiny)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--impl", "reference", "--workload", "fwd_fp8_tiny", "--steps", "1", "--warmup", "1"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.FP8_METRIC and line["value"] > 0
 
 
 def test_decode_workload_bytes():
