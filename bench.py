@@ -52,7 +52,7 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--e2e-steps", type=int, default=8)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args(argv)
@@ -137,59 +137,155 @@ def captured_traffic(kernel: str, workload: str):
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and clock-event (throttle) reasons while the timed
+    region runs. Polls NVML from a thread every ~5 ms (read-only queries;
+    nothing is set), falling back to ``nvidia-smi -lms 20``; the summary keeps
+    only the samples taken between ``begin()`` and ``end()`` (host time),
+    and the nearest one if the region is shorter than the polling period."""
 
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device):
+        self.device = device
+        self.samples = []  # (host time, sm MHz, max sm MHz, set of reason names)
+        self.t_begin = self.t_end = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
 
-    def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
-                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
-        return self
+    def _nvml_handle(self):
+        import pynvml
+        import torch
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.device)
+        bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.thread.join(timeout=2)
+    def _poll_nvml(self, pynvml, h):
+        reasons_of = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or getattr(
+            pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            bits = reasons_of(h)
+            names = {n for b, n in self.REASONS.items() if bits & b}
+            self.samples.append((time.monotonic(), float(sm), float(mx), names))
+            self._stop.wait(0.005)
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+    def _poll_smi(self):
+        for line in self._proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+            names = {n for n, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                      parts[5:9]) if v.lower() == "active"}
+            self.samples.append((time.monotonic(), sm, mx, names))
+
+    def __enter__(self):
+        try:
+            pynvml, h = self._nvml_handle()
+            self._thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h), daemon=True)
+        except Exception:
+            try:
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                     "-i", str(self.device.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self._thread = threading.Thread(target=self._poll_smi, daemon=True)
+            except OSError:
+                self._thread = None
+        if self._thread is not None:
+            self._thread.start()
+        return self
+
+    def begin(self):
+        self.t_begin = time.monotonic()
+
+    def end(self):
+        self.t_end = time.monotonic()
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        b = self.t_begin if self.t_begin is not None else self.samples[0][0]
+        e = self.t_end if self.t_end is not None else self.samples[-1][0]
+        inside = [x for x in self.samples if b <= x[0] <= e]
+        if not inside:  # region shorter than the polling period: the sample nearest its middle
+            mid = 0.5 * (b + e)
+            inside = [min(self.samples, key=lambda x: abs(x[0] - mid))]
+        reasons = set().union(*(x[3] for x in inside))
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ------------------------------------------------------ end to end
+
+def pipelined_e2e(dev, compute_stream, host_in, make_set, run, steps):
+    """Times ``steps`` end-to-end steps through the public API, pipelined the
+    way a caller streaming batches would: two sets of device buffers
+    alternate; step k copies its inputs from pinned host memory into set k % 2
+    on a copy-in stream, computes on ``compute_stream`` once they are in, and
+    copies every output back to pinned host memory on a copy-out stream, so
+    that the next step's inputs and the previous step's outputs cross the
+    host link while this step computes (in both directions at once). Every
+    step moves all its input and output bytes. Returns the device time in ms
+    from the first copy-in to the last copy-out.
+
+    ``make_set()`` returns (device inputs in the order of ``host_in``, device
+    outputs); ``run(dev_in, dev_out, stream)`` enqueues one step's compute."""
+    import torch
+
+    sets = [make_set() for _ in range(2)]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs] for _, outs in sets]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    in_done = [ev() for _ in range(steps)]
+    comp_done = [ev() for _ in range(steps)]
+    out_done = [ev() for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(s_in)
+    for k in range(steps):
+        dins, douts = sets[k % 2]
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(comp_done[k - 2])  # set k % 2's inputs were read by step k - 2
+            for d, h in zip(dins, host_in):
+                d.copy_(h, non_blocking=True)
+            in_done[k].record(s_in)
+        compute_stream.wait_event(in_done[k])
+        if k >= 2:
+            compute_stream.wait_event(out_done[k - 2])  # set k % 2's outputs were copied out
+        run(dins, douts, compute_stream)
+        comp_done[k].record(compute_stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[k])
+            for h, d in zip(host_out[k % 2], douts):
+                h.copy_(d, non_blocking=True)
+            out_done[k].record(s_out)
+    s_out.wait_event(out_done[steps - 1])
+    t1.record(s_out)
+    torch.cuda.synchronize(dev)
+    return t0.elapsed_time(t1)
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -421,8 +517,9 @@ def native_arm(args):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clocks:
-        time.sleep(0.3)
+    with ClockSampler(dev) as clocks:
+        time.sleep(0.05)
+        clocks.begin()
         t_start.record(stream)
         for s in range(args.steps):
             if w.backward:
@@ -430,6 +527,7 @@ def native_arm(args):
             step(evs[s])
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.end()
     fa.fa_profile_set_bwd_events(None, None)
     barrier(dev)
     if fa.fa_check_device_error(stream) != fa.FA_OK:
@@ -465,37 +563,35 @@ def native_arm(args):
     }
 
     # End to end through the public API: pinned host inputs copied in, both
-    # passes run, every output copied back, all inside the timed region.
+    # passes run, every output copied back, all inside the timed region
+    # (pipelined across steps, see pipelined_e2e).
     e2e = None
     if args.e2e_steps > 0:
-        hin = {n: host[n].pin_memory() for n in host}
-        outs = [o, lse] + ([dq, dk, dv] if w.backward else [])
-        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-        h2d = sum(t.numel() * t.element_size() for t in hin.values())
-        d2h = sum(t.numel() * t.element_size() for t in outs)
-        dins = {"q": q, "k": k, "v": v}
-        if w.backward:
-            dins["dout"] = dout
+        names = ["q", "k", "v"] + (["dout"] if w.backward else [])
+        hin = [host[n].pin_memory() for n in names]
 
-        def e2e_step():
-            for n, t in dins.items():
-                t.copy_(hin[n], non_blocking=True)
-            step()
-            for src, dst in zip(outs, hout):
-                dst.copy_(src, non_blocking=True)
+        def make_set():
+            dins = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hin]
+            douts = [torch.empty_like(o), torch.empty_like(lse)]
+            if w.backward:
+                douts += [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+            return dins, douts
 
-        e2e_step()
-        torch.cuda.synchronize(dev)
+        def run(dins, douts, st):
+            eq, ek, ev_ = dins[0], dins[1], dins[2]
+            fa.fa_fwd(eq, ek, ev_, douts[0], douts[1], w.causal, w.scale, st, o_resid=o_resid)
+            if w.backward:
+                fa.fa_bwd(eq, ek, ev_, douts[0], dins[3], douts[1], douts[2], douts[3], douts[4], w.causal,
+                          w.scale, ws, st, o_resid=o_resid)
+
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = sum(t.numel() * t.element_size() for t in [o, lse] + ([q, k, v] if w.backward else []))
+        pipelined_e2e(dev, stream, hin, make_set, run, 2)  # warm-up of the streams and buffers
         barrier(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e_ms = max_over_ranks(pipelined_e2e(dev, stream, hin, make_set, run, args.e2e_steps), dev)
         e2e = {"value": step_flops * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipelined": "inputs of step k+1 and outputs of step k-1 cross the host link while step k computes"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -562,13 +658,15 @@ def fp8_native_arm(args, w):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clocks:
-        time.sleep(0.3)
+    with ClockSampler(dev) as clocks:
+        time.sleep(0.05)
+        clocks.begin()
         t_start.record(stream)
         for _ in range(args.steps):
             step()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.end()
     barrier(dev)
     if fa.fa_check_device_error(stream) != fa.FA_OK:
         raise RuntimeError("device watchdog fired during the timed steps")
@@ -679,8 +777,9 @@ def decode_native_arm(args, w):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clocks:
-        time.sleep(0.3)
+    with ClockSampler(dev) as clocks:
+        time.sleep(0.05)
+        clocks.begin()
         t_start.record(stream)
         for s in range(args.steps):
             evs[s][0].record(stream)
@@ -689,6 +788,7 @@ def decode_native_arm(args, w):
             evs[s][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.end()
     fa.fa_profile_set_decode_event(None)
     barrier(dev)
     if fa.fa_check_device_error(stream) != fa.FA_OK:

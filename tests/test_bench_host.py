@@ -124,3 +124,15 @@ def test_captured_traffic_requires_unchanged_sources(tmp_path, monkeypatch):
     assert bench.captured_traffic("kern", "other") is None
     (csrc / "k.cu").write_bytes(b"kernel source v2")
     assert bench.captured_traffic("kern", "wl") is None
+
+
+def test_clock_summary_keeps_only_the_timed_window():
+    c = bench.ClockSampler(None)
+    c.samples = [(0.0, 1200.0, 1965.0, set()), (1.0, 1965.0, 1965.0, {"sw_power_cap"}),
+                 (1.5, 1900.0, 1965.0, set()), (3.0, 800.0, 1965.0, {"hw_slowdown"})]
+    c.t_begin, c.t_end = 0.9, 2.0
+    sm = c.summary()
+    assert sm["samples"] == 2 and sm["sm_mhz"] == (1965.0 + 1900.0) / 2
+    assert sm["reasons"] == ["sw_power_cap"] and sm["sm_max_mhz"] == 1965.0
+    c.t_begin, c.t_end = 2.1, 2.2  # shorter than the polling period: nearest sample to its middle
+    assert c.summary()["samples"] == 1 and c.summary()["sm_mhz"] == 1900.0
