@@ -138,7 +138,7 @@ def captured_traffic(kernel: str, workload: str):
 
 class ClockSampler:
     """Samples SM clocks and clock-event (throttle) reasons while the timed
-    region runs. Polls NVML from a thread every ~5 ms (read-only queries;
+    region runs. Polls NVML from a thread every ~1 ms (read-only queries;
     nothing is set), falling back to ``nvidia-smi -lms 20``; the summary keeps
     only the samples taken between ``begin()`` and ``end()`` (host time),
     and the nearest one if the region is shorter than the polling period."""
@@ -164,7 +164,14 @@ class ClockSampler:
         pynvml.nvmlInit()
         p = torch.cuda.get_device_properties(self.device)
         bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
-        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        for arg in (bus, bus.encode()):
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(arg)
+            except Exception:
+                pass
+        if "CUDA_VISIBLE_DEVICES" not in os.environ:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device.index)
+        raise RuntimeError(f"no NVML device with PCI bus id {bus}")
 
     def _poll_nvml(self, pynvml, h):
         reasons_of = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or getattr(
@@ -175,7 +182,7 @@ class ClockSampler:
             bits = reasons_of(h)
             names = {n for b, n in self.REASONS.items() if bits & b}
             self.samples.append((time.monotonic(), float(sm), float(mx), names))
-            self._stop.wait(0.005)
+            self._stop.wait(0.001)
 
     def _poll_smi(self):
         for line in self._proc.stdout:
@@ -194,7 +201,8 @@ class ClockSampler:
         try:
             pynvml, h = self._nvml_handle()
             self._thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h), daemon=True)
-        except Exception:
+        except Exception as exc:
+            print(f"bench.py: NVML clock sampling unavailable ({exc}); using nvidia-smi", file=sys.stderr)
             try:
                 self._proc = subprocess.Popen(
                     ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
@@ -207,6 +215,10 @@ class ClockSampler:
         return self
 
     def begin(self):
+        # The sampler must be running before the timed region starts.
+        t0 = time.monotonic()
+        while not self.samples and self._thread is not None and time.monotonic() - t0 < 3.0:
+            time.sleep(0.01)
         self.t_begin = time.monotonic()
 
     def end(self):
