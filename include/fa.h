@@ -67,6 +67,11 @@ extern "C" {
  *   o [B][Hq][N][d] (bf16, written), lse [B][Hq][N] (fp32, written)
  *   causal: 0 or 1 (query i sees keys j <= i)
  *   stream: cudaStream_t or NULL
+ * Rounding: a row's running max is refreshed (and O rescaled) only when it
+ * grows by more than 8 in log2 units, so softmax weights reach 2^8 before
+ * normalisation and the row's largest weight enters the P v product as a
+ * bf16-rounded 2^delta rather than exactly 1 (relative error <= 2^-9, the
+ * same as any other weight); lse is formed from unrounded weights.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
            int d, int causal, float scale, void* stream);
@@ -74,7 +79,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 /*
  * Forward pass that also writes the bf16 rounding residual of o:
  * o_resid = bf16(O - o), where O is the fp32 result before rounding and o is
- * what fa_fwd writes. o + o_resid carries O to ~16 significant bits.
+ * its bf16 rounding. o + o_resid carries O to ~16 significant bits. This
+ * forward refreshes a row's running max whenever it grows, so the largest
+ * weight of every row enters P v as exactly 1; its o may differ from
+ * fa_fwd's in the last bit.
  * fa_bwd_with_residual uses it to form D_i = sum_c dO_ic O_ic: D multiplies
  * every error of O by dO and sums it over d, so the bf16 rounding of o alone
  * shifts dQ and dK by ~1e-2 on peaky rows. Arguments as fa_fwd, plus
