@@ -382,10 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int q0 = c * 32 + 4 * y;
           const float4 lq = *reinterpret_cast<const float4*>(l2 + q0);
           const float4 dq = *reinterpret_cast<const float4*>(dd + q0);
-          float p[4] = {ex2(fmaf(__uint_as_float(sv[4 * y]), sl2, -lq.x)),
-                        ex2(fmaf(__uint_as_float(sv[4 * y + 1]), sl2, -lq.y)),
-                        ex2(fmaf(__uint_as_float(sv[4 * y + 2]), sl2, -lq.z)),
-                        ex2(fmaf(__uint_as_float(sv[4 * y + 3]), sl2, -lq.w))};
+          // Exponent arguments, dP - D and the products two at a time
+          // (packed f32x2, same rounding as the scalar form).
+          float p[4];
+          ffma2(p[0], p[1], __uint_as_float(sv[4 * y]), __uint_as_float(sv[4 * y + 1]), sl2, sl2, -lq.x, -lq.y);
+          ffma2(p[2], p[3], __uint_as_float(sv[4 * y + 2]), __uint_as_float(sv[4 * y + 3]), sl2, sl2, -lq.z, -lq.w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) p[e] = ex2(p[e]);
           if (q0 < diag_lim) {
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -398,10 +401,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!((key <= qg && qg - key <= a.window) || key < a.prefix)) p[e] = 0.f;
             }
           }
-          const float g0 = p[0] * (__uint_as_float(dv[4 * y]) - dq.x);
-          const float g1 = p[1] * (__uint_as_float(dv[4 * y + 1]) - dq.y);
-          const float g2 = p[2] * (__uint_as_float(dv[4 * y + 2]) - dq.z);
-          const float g3 = p[3] * (__uint_as_float(dv[4 * y + 3]) - dq.w);
+          float g0, g1, g2, g3;
+          fsub2(g0, g1, __uint_as_float(dv[4 * y]), __uint_as_float(dv[4 * y + 1]), dq.x, dq.y);
+          fsub2(g2, g3, __uint_as_float(dv[4 * y + 2]), __uint_as_float(dv[4 * y + 3]), dq.z, dq.w);
+          fmul2(g0, g1, p[0], p[1], g0, g1);
+          fmul2(g2, g3, p[2], p[3], g2, g3);
           pk[2 * y] = pack_bf16x2(p[0], p[1]);
           pk[2 * y + 1] = pack_bf16x2(p[2], p[3]);
           dk[2 * y] = pack_bf16x2(g0, g1);

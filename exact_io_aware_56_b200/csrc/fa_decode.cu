@@ -386,10 +386,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), sl2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, neg_m));
-          ps[(2 * i) & 7] += p0;
-          ps[(2 * i + 1) & 7] += p1;
+          // Exponent arguments and partial sums two at a time (packed f32x2).
+          float x0, x1;
+          ffma2(x0, x1, __uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, sl2,
+                neg_m, neg_m);
+          const float p0 = ex2(x0);
+          const float p1 = ex2(x1);
+          fadd2(ps[(2 * i) & 7], ps[(2 * i + 1) & 7], ps[(2 * i) & 7], ps[(2 * i + 1) & 7], p0, p1);
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tP + cp * (CW / 2) + c * 16, pk);
@@ -404,7 +407,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           uint32_t o32[32];
           tmem_ld32(tO + c * 32, o32);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            fmul2(x0, x1, __uint_as_float(o32[i]), __uint_as_float(o32[i + 1]), alpha, alpha);
+            o32[i] = __float_as_uint(x0);
+            o32[i + 1] = __float_as_uint(x1);
+          }
           tmem_st32(tO + c * 32, o32);
         }
       }

@@ -123,7 +123,7 @@ struct FwdArgs {
 struct FwdBars {
   uint64_t q_full;
   uint64_t k_full[4], v_full[4], kv_empty[4];
-  uint64_t s_full[2], p_ready[2], o_final[2];
+  uint64_t s_full[2], p_ready[2][2], o_final[2];  // p_ready: [Q tile][half of P]
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_ready[t], kBM);
+      mbar_init(&bars->p_ready[t][0], kBM);
+      mbar_init(&bars->p_ready[t][1], kBM);
       mbar_init(&bars->o_final[t], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -282,12 +283,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars->s_full[t]);
       };
-      auto issue_pv = [&](int t, int j) {
+      // Half h of P V: keys [64h, 64h + 64).
+      auto issue_pv = [&](int t, int j, int h) {
         const uint32_t va = sV + (j % ST) * C::kTileBytes;
         // P: KS keys per step = 8 tensor-memory columns (bf16 pairs or e4m3
         // quads); V: KS key rows of 128 bytes (MN-major).
+        constexpr int KH = kBN / KS / 2;
 #pragma unroll
-        for (int k = 0; k < kBN / KS; ++k) {
+        for (int k = h * KH; k < h * KH + KH; ++k) {
           if constexpr (F8)
             mma_ts_f8(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * KS * 128, C::kBoxBytes, 1024), idesc_pv,
                       (j > 0 || k > 0) ? 1u : 0u);
@@ -308,18 +311,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t par = (j / ST) & 1;
         const int jn = j + 1;
         if (j < n0) {
-          if (!(ok = wait_bar(&bars->p_ready[0], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
+          if (!(ok = wait_bar(&bars->p_ready[0][0], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
           tc_fence_after();
-          issue_pv(0, j);
+          issue_pv(0, j, 0);
+          if (!(ok = wait_bar(&bars->p_ready[0][1], j & 1, w))) break;
+          tc_fence_after();
+          issue_pv(0, j, 1);
           if (j == n0 - 1) mma_commit(&bars->o_final[0]);
           if (jn < n0) {
             if (!(ok = wait_bar(&bars->k_full[jn % ST], (jn / ST) & 1, w))) break;
             issue_s(0, jn);
           }
         }
-        if (!(ok = wait_bar(&bars->p_ready[1], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
+        if (!(ok = wait_bar(&bars->p_ready[1][0], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
         tc_fence_after();
-        issue_pv(1, j);
+        issue_pv(1, j, 0);
+        if (!(ok = wait_bar(&bars->p_ready[1][1], j & 1, w))) break;
+        tc_fence_after();
+        issue_pv(1, j, 1);
         mma_commit(&bars->kv_empty[s]);
         if (j == n1 - 1) mma_commit(&bars->o_final[1]);
         if (jn < n1) {
@@ -416,10 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       float ps[8];  // 8 independent partial row sums
 #pragma unroll
       for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-      if constexpr (F8) {
-        // 64 scores -> 16 columns of four e4m3 each.
+      // P goes to tensor memory in two halves of 64 keys. The first half is
+      // released to the MMA thread (after the O rescale, which must precede
+      // any of this tile's P V) while the second half's exponentials run, so
+      // half of P V overlaps the softmax.
 #pragma unroll
-        for (int c = 0; c < kBN / 64; ++c) {
+      for (int h = 0; h < 2; ++h) {
+        if constexpr (F8) {
+          // 64 scores -> 16 columns of four e4m3 each.
+          const int c = h;
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -437,41 +451,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[i] = pack_e4m3x4(p4[0], p4[1], p4[2], p4[3]);
           }
           tmem_st16(tS + c * 16, pk);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            // Exponent arguments and partial sums two at a time (packed
-            // f32x2: half the FMA and add instructions of the scalar form).
-            float x0, x1;
-            ffma2(x0, x1, __uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1]), sl2, sl2,
-                  neg_m, neg_m);
-            const float p0 = (2 * i < kPolyPer32) ? exp2_poly(x0) : ex2(x0);
-            const float p1 = (2 * i + 1 < kPolyPer32) ? exp2_poly(x1) : ex2(x1);
-            fadd2(ps[(2 * i) & 7], ps[(2 * i + 1) & 7], ps[(2 * i) & 7], ps[(2 * i + 1) & 7], p0, p1);
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
-      }
-      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      if (rescale) {
-        // O holds every earlier product (see the ordering argument above);
-        // scale this row by alpha before P V is added to it.
-        if constexpr (D == 128) {
-          uint32_t ov[128];
-          tmem_ld128(tO, ov);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o32[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(ov[c * 32 + i]) * alpha);
-            tmem_st32(tO + c * 32, o32);
-          }
         } else {
+#pragma unroll
+          for (int c = 2 * h; c < 2 * h + 2; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              // Exponent arguments and partial sums two at a time (packed
+              // f32x2: half the FMA and add instructions of the scalar form).
+              float x0, x1;
+              ffma2(x0, x1, __uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1]), sl2,
+                    sl2, neg_m, neg_m);
+              const float p0 = (2 * i < kPolyPer32) ? exp2_poly(x0) : ex2(x0);
+              const float p1 = (2 * i + 1 < kPolyPer32) ? exp2_poly(x1) : ex2(x1);
+              fadd2(ps[(2 * i) & 7], ps[(2 * i + 1) & 7], ps[(2 * i) & 7], ps[(2 * i + 1) & 7], p0, p1);
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + c * 16, pk);
+          }
+        }
+        if (h == 0 && rescale) {
+          // O holds every earlier product (see the ordering argument above);
+          // scale this row by alpha before P V is added to it.
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o32[32];
@@ -481,11 +482,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + c * 32, o32);
           }
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready[t][h]);
       }
-      l += sum;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->p_ready[t]);
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->o_final[t], 0, w));
     if (ok) {
