@@ -20,17 +20,20 @@
 //   warps 10-11 idle (keep the third warpgroup whole).
 // The softmax is the online form of the "Four ideas" list (item "Online
 // softmax"): running max m, running sum l, O rescaled by e^(m - m_new)
-// when the max grows.
+// when the max grows (by more than the rescale threshold below). P_t goes
+// back to the MMA thread in two halves of 64 keys, one barrier each; the O
+// rescale precedes the first, and the first half's share of O_t += P_t V_j
+// runs while the second half's exponentials are computed.
 //
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [0,128) S_0 | [128,256) S_1 | [256,256+D) O_0 | [256+D,256+2D) O_1
 // P_t (bf16, two per column) overwrites the first 64 columns of S_t.
 //
 // Ordering argument used by the softmax warps: the MMA thread issues, for
-// each tile t, S_t^(j+1) after O_t += P_t^j V_j, and tcgen05 operations
-// complete in issue order, so once S_t^(j+1) is signalled complete the O_t
-// accumulator holds every earlier product and may be rescaled in place
-// until P_t^(j+1) is handed back.
+// each tile t, S_t^(j+1) after both halves of O_t += P_t^j V_j, and tcgen05
+// operations complete in issue order, so once S_t^(j+1) is signalled
+// complete the O_t accumulator holds every earlier product and may be
+// rescaled in place until the first half of P_t^(j+1) is handed back.
 //
 // The exponentials are base 2: scores are scaled by scale*log2(e), and
 // L = (m + log2 l) * ln 2. A warp whose rows' maxima did not grow on a tile
