@@ -3,8 +3,10 @@
 import math
 
 import numpy as np
+import pytest
 
 import oracle
+from oracle import attention as A
 
 from .test_oracle_pins import rnd
 
@@ -35,3 +37,57 @@ def test_decode_zero_query_is_mean_of_cache():
     O, L = oracle.attn_decode_ref(np.zeros((1, 1, 1, 4)), rnd((1, 1, 17, 4), 322), v, 1.0)
     np.testing.assert_allclose(O[0, 0, 0], v[0, 0].mean(0), atol=1e-15)
     assert abs(L[0, 0, 0] - math.log(17)) < 1e-15
+
+
+# --------------------------------------------------------------- mutations
+# Planted mistakes in the decode oracle (CPU only): each must make at least
+# one of the pins above fail.
+
+PINS = [test_decode_equals_last_rows_of_full_causal, test_single_query_sees_every_key_brute_force,
+        test_decode_zero_query_is_mean_of_cache]
+
+
+def _mutated_decode(kind):
+    def decode(q, k, v, scale, causal=True):
+        B, Hq, Nq, d = q.shape
+        Hkv, Nk = k.shape[1], k.shape[2]
+        pos = np.arange(Nk - Nq, Nk)
+        if kind == "top-left alignment":
+            pos = np.arange(Nq)
+        elif kind == "alignment off by one":
+            pos = pos - 1
+        O = np.empty((B, Hq, Nq, d))
+        L = np.empty((B, Hq, Nq))
+        for b in range(B):
+            for h in range(Hq):
+                g = h % Hkv if kind == "kv head by modulo" else A.kv_head_of(h, Hq, Hkv)
+                S = A._scores(q[b, h], k[b, g], 1.0 if kind == "scale dropped" else scale, causal, pos)
+                P, Lr = A._softmax_rows(S)
+                if kind == "not normalised":
+                    P = np.exp(S - S.max(axis=1, keepdims=True))
+                O[b, h] = P @ v[b, g]
+                L[b, h] = Lr
+        return O, L
+    return decode
+
+
+def _some_pin_fails():
+    for pin in PINS:
+        try:
+            pin()
+        except AssertionError:
+            return True
+    return False
+
+
+@pytest.mark.parametrize("kind", ["top-left alignment", "alignment off by one", "kv head by modulo",
+                                  "scale dropped", "not normalised"])
+def test_decode_mutation_is_caught(monkeypatch, kind):
+    monkeypatch.setattr(oracle, "attn_decode_ref", _mutated_decode(kind))
+    assert _some_pin_fails(), kind
+
+
+def test_unmutated_decode_reimplementation_passes(monkeypatch):
+    # The mutation harness itself, with no mutation, passes every pin.
+    monkeypatch.setattr(oracle, "attn_decode_ref", _mutated_decode("none"))
+    assert not _some_pin_fails()
