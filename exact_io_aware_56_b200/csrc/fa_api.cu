@@ -380,6 +380,17 @@ int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* strea
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
 
+int fa_test_decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas, long long* out) {
+  if (!out || num_ctas < 1) return FA_ERR_INVALID_ARGUMENT;
+  const int rc = check_decode_shape(B, Hq, Hkv, Nq, Nk, d, 0, 1.f);
+  if (rc != FA_OK) return rc;
+  const DecodeShape s{B, Hq, Hkv, Nq, Nk, d, 0, 1.f};
+  const DecodePlan p = make_decode_plan(s, num_ctas);
+  const long long v[8] = {p.W, p.T, p.G, p.MS, p.R, p.rho, p.rv, p.n_chunks};
+  for (int i = 0; i < 8; ++i) out[i] = v[i];
+  return FA_OK;
+}
+
 void fa_profile_set_decode_event(void* after_main) { g_ev_dec.store(after_main); }
 
 void fa_profile_set_bwd_events(void* after_pre, void* after_main) {

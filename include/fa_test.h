@@ -32,6 +32,19 @@ void fa_test_set_fault(int code);
  */
 int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* stream);
 
+/*
+ * Host only (no device call): the stream-K work partition fa_decode would
+ * use for this shape with num_ctas CTAs, as eight integers in out[0..7]:
+ * W (key tiles over all units), T (128-key tiles per unit), G (CTAs = runs),
+ * MS (most units one run may touch), R (query rows per KV head), rho (row
+ * replication over the 128 tensor-memory lanes), rv (stored rows per copy),
+ * n_chunks (row chunks per KV head). A unit is (batch, KV head, row chunk);
+ * run c covers tiles [c*W/G, (c+1)*W/G) in unit order. Returns FA_OK,
+ * FA_ERR_INVALID_ARGUMENT (null out, num_ctas < 1, bad shape) or
+ * FA_ERR_UNSUPPORTED, as fa_decode would for the shape.
+ */
+int fa_test_decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas, long long* out);
+
 #ifdef __cplusplus
 }
 #endif
