@@ -175,8 +175,10 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
  * (the prefix tiles and the window tiles, skipping any gap between them).
  * Arguments as fa_fwd_with_residual / fa_bwd_with_residual, with the causal
  * flag replaced by (window, prefix); o_resid may be NULL in both (the
- * backward then forms D from o alone). FA_ERR_INVALID_ARGUMENT when
- * window < -1 or prefix < 0.
+ * backward then forms D from o alone). Without o_resid the forward rounds
+ * as fa_fwd does (deferred O rescale), with it as fa_fwd_with_residual
+ * (exact running max). FA_ERR_INVALID_ARGUMENT when window < -1 or
+ * prefix < 0.
  */
 int fa_fwd_masked(const void* q, const void* k, const void* v, void* o, void* o_resid, float* lse, int B, int Hq,
                   int Hkv, int N, int d, int window, int prefix, float scale, void* stream);
