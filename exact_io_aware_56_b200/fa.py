@@ -93,6 +93,10 @@ def _check_tensor(name, t, dtype, shape):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise RuntimeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.get_device() != torch.cuda.current_device():
+        # The library launches on the current device with raw pointers.
+        raise ValueError(f"{name} is on cuda:{t.get_device()} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if tuple(t.shape) != tuple(shape):
