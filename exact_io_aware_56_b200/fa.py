@@ -106,6 +106,14 @@ def _check_tensor(name, t, dtype, shape):
     return t.data_ptr()
 
 
+def _check_workspace(workspace):
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if workspace.get_device() != torch.cuda.current_device():
+        raise ValueError(f"workspace is on cuda:{workspace.get_device()} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+
+
 def _shapes(q, k):
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q and k must be [B, H, N, d]")
@@ -166,8 +174,7 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal: bool, scale: float, worksp
             _check_tensor("lse", lse, torch.float32, (B, Hq, N)),
             _check_tensor("dq", dq, bf, (B, Hq, N, d)), _check_tensor("dk", dk, bf, (B, Hkv, N, d)),
             _check_tensor("dv", dv, bf, (B, Hkv, N, d))]
-    if not workspace.is_cuda or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check_workspace(workspace)
     ws_bytes = workspace.numel() * workspace.element_size()
     mask = _mask_args(causal, window, prefix)
     tail = (B, Hq, Hkv, N, d, int(bool(causal)), float(scale), workspace.data_ptr(), ws_bytes, _stream(stream))
@@ -233,8 +240,7 @@ def fa_decode(q, k, v, o, lse, causal: bool, scale: float, workspace, stream=Non
     args = [_check_tensor("q", q, bf, (B, Hq, Nq, d)), _check_tensor("k", k, bf, (B, Hkv, Nk, d)),
             _check_tensor("v", v, bf, (B, Hkv, Nk, d)), _check_tensor("o", o, bf, (B, Hq, Nq, d)),
             _check_tensor("lse", lse, torch.float32, (B, Hq, Nq))]
-    if not workspace.is_cuda or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check_workspace(workspace)
     rc = lib().fa_decode(*args, B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale), workspace.data_ptr(),
                          workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != FA_OK:
