@@ -94,3 +94,53 @@ def test_workspace_size_formula(L):
     assert n < B * Hq * N * 4 + B * Hq * N * d * 4 + (1 << 20)
     assert L.fa_bwd_workspace_bytes(1, 1, 1, 16, 96) == 0
     assert L.fa_bwd_workspace_bytes(0, 1, 1, 16, 64) == 0
+
+
+def test_other_entry_points_reject_bad_arguments_before_launch(L):
+    p = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: rejected before use
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    INV, UNS = fa.FA_ERR_INVALID_ARGUMENT, fa.FA_ERR_UNSUPPORTED
+
+    # Masked forward / backward: window < -1 or prefix < 0 is invalid.
+    def fwdm(q=p, window=-1, prefix=0, d=64):
+        return L.fa_fwd_masked(q, p, p, p, None, p, 1, 2, 1, 16, d, window, prefix, 0.125, None)
+
+    assert fwdm(window=-2) == INV and fwdm(prefix=-1) == INV and fwdm(q=None) == INV and fwdm(d=96) == UNS
+
+    def bwdm(window=-1, prefix=0, ws_bytes=1 << 30):
+        return L.fa_bwd_masked(p, p, p, p, None, p, p, p, p, p, 1, 2, 1, 16, 64, window, prefix, 0.125, p,
+                               ws_bytes, None)
+
+    assert bwdm(window=-5) == INV and bwdm(prefix=-3) == INV and bwdm(ws_bytes=8) == INV
+
+    # FP8 quantizer and forward.
+    def quant(x=p, scales=p, BH=2, N=16, d=64, per_head=0):
+        return L.fa_quantize_fp8(x, p, scales, BH, N, d, per_head, None)
+
+    assert quant(x=None) == INV and quant(x=mis) == INV and quant(scales=ctypes.c_void_p((1 << 20) + 2)) == INV
+    assert quant(BH=0) == INV and quant(N=-1) == INV and quant(per_head=2) == INV and quant(d=96) == UNS
+
+    def fwd8(sq=p, d=128, Hq=2, Hkv=1, scale=0.1):
+        return L.fa_fwd_fp8(p, sq, p, p, p, p, p, p, 1, Hq, Hkv, 16, d, 1, scale, None)
+
+    assert fwd8(sq=None) == INV and fwd8(sq=ctypes.c_void_p((1 << 20) + 1)) == INV
+    assert fwd8(scale=float("inf")) == INV and fwd8(d=64) == UNS and fwd8(Hq=3, Hkv=2) == UNS
+
+    # Decode.
+    def dec(q=p, Nq=1, Nk=16, d=64, ws_bytes=1 << 30, Hq=2, Hkv=1):
+        return L.fa_decode(q, p, p, p, p, 1, Hq, Hkv, Nq, Nk, d, 1, 0.125, p, ws_bytes, None)
+
+    assert dec(q=None) == INV and dec(q=mis) == INV and dec(Nq=17) == INV and dec(Nk=0) == INV
+    assert dec(d=96) == UNS and dec(Hq=3, Hkv=2) == UNS and dec(ws_bytes=8) == INV
+    assert L.fa_decode_workspace_bytes(1, 2, 1, 17, 16, 64) == 0
+    assert L.fa_decode_workspace_bytes(1, 2, 1, 1, 16, 96) == 0
+    assert L.fa_decode_workspace_bytes(1, 2, 1, 1, 16, 64) > 0
+
+    # No-allocation backward: shapes it cannot hold are rejected before any CUDA call.
+    L.fa_bwd_noalloc.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 + [ctypes.c_float, ctypes.c_void_p]
+    L.fa_bwd_noalloc.restype = ctypes.c_int
+
+    def bwdn(B=1, N=16, d=64):
+        return L.fa_bwd_noalloc(p, p, p, p, p, p, p, p, p, B, 2, 1, N, d, 1, 0.125, None)
+
+    assert bwdn(B=0) == INV and bwdn(d=96) == UNS and bwdn(N=1 << 20) == UNS
