@@ -26,6 +26,8 @@ none is "parity unpinned".
 from .attention import (  # noqa: F401
     attn_fwd_ref,
     attn_fwd_online_ref,
+    merge_softmax_states,
+    softmax_state,
     attn_bwd_ref,
     attn_fwd_rows,
     attn_bwd_rows,

@@ -126,23 +126,70 @@ def attn_fwd_ref(q, k, v, causal: bool, scale: float, window=None, prefix=0):
     return O, L
 
 
-def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
-                        block_q: int = 128, block_k: int = 128, window=None, prefix=0):
-    """Tiled forward with the online softmax, in the pages' order.
+def softmax_state(S, V):
+    """Partial softmax state of one block of keys for each query row.
 
-    FlashAttention: IO-aware exact attention, "FLASH" box of the "NAIVE
-    ATTENTION vs FLASHATTENTION" diagram: for each Q block start from
-    O = 0, m = -inf, l = 0; for each K, V block form the score tile, raise
-    the running max, rescale l and O by e^(m - m_new), add the new block's
-    exponentials, and move m forward. After the last block O is divided by
-    l and L = m + ln l is kept (the box's final line; the divide is the
-    plain reading of "write O once"). Only m, l and O persist between
-    blocks ("PREFILL PATH" diagram: "Only m, l, O stay"); no N x N array is
-    built. Returns ``(O, L)`` like :func:`attn_fwd_ref`.
+    For score rows ``S`` [rows, keys] (masked entries -inf) and the block's
+    values ``V`` [keys, d] the state is (m, l, U): the row max m of S, the
+    sum l of exp(S - m) and the unnormalised output U = exp(S - m) V. A row
+    with every key of the block masked has m = -inf, l = 0 and U = 0 (the
+    empty state). The normalised output of the block alone is U / l.
+    """
+    m = S.max(axis=1)
+    ref = np.where(np.isneginf(m), 0.0, m)
+    E = np.exp(S - ref[:, None])
+    return m, E.sum(axis=1), E @ V
+
+
+def merge_softmax_states(a, b):
+    """Softmax state over the union of two disjoint key sets.
+
+    FlashAttention: IO-aware exact attention, "Four ideas" list, item
+    "Online softmax": a partial output is rescaled to a new, larger maximum
+    and the rescale is exact; Flash Attention: memory-efficient
+    transformers, "Online Softmax": the normalisation is updated per block
+    instead of in a second pass. Written as the identity behind both: with
+    M = max(m_a, m_b), sum_j exp(S_j - M) splits over the two key sets as
+    e^(m_a - M) l_a + e^(m_b - M) l_b, and likewise for U. The operation
+    is associative and commutative (up to rounding), so any order of
+    merging gives the softmax over all keys. Empty states (m = -inf)
+    contribute nothing.
+    """
+    ma, la, Ua = a
+    mb, lb, Ub = b
+    M = np.maximum(ma, mb)
+    ref = np.where(np.isneginf(M), 0.0, M)
+    fa = np.where(np.isneginf(ma), 0.0, np.exp(ma - ref))
+    fb = np.where(np.isneginf(mb), 0.0, np.exp(mb - ref))
+    return M, fa * la + fb * lb, fa[:, None] * Ua + fb[:, None] * Ub
+
+
+def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
+                        block_q: int = 128, block_k: int = 128, window=None, prefix=0, order=None):
+    """Tiled forward built from per-block softmax states and their merge.
+
+    Each (query block, key block) pair yields its own softmax state
+    (:func:`softmax_state`); a query block's states over all key blocks are
+    combined by :func:`merge_softmax_states`, so no N x N array is ever
+    built and only (m, l, U) of a query block persist between key blocks
+    (FlashAttention: IO-aware exact attention, "PREFILL PATH" diagram: only
+    m, l and O stay on chip). The result is O = U / l and the row logsumexp
+    L = m + ln l (natural log; the pages keep one logsumexp per query row).
+
+    ``order`` (optional) is a permutation of the key-block indices giving the
+    order in which states are merged, left to right; by default they are
+    merged in ascending order, the order of a kernel streaming K/V blocks.
+    Since the merge is associative and commutative, every order must give
+    the two-pass result. Returns ``(O, L)`` like :func:`attn_fwd_ref`.
     """
     B, Hq, Hkv, N, d = _check(q, k, v)
     if block_q < 1 or block_k < 1:
         raise ValueError("block sizes must be positive")
+    starts = list(range(0, N, block_k))
+    if order is None:
+        order = range(len(starts))
+    elif sorted(order) != list(range(len(starts))):
+        raise ValueError("order must be a permutation of the key-block indices")
     O_out = np.empty_like(q, dtype=np.float64)
     L_out = np.empty((B, Hq, N), dtype=np.float64)
     for b in range(B):
@@ -150,25 +197,15 @@ def attn_fwd_online_ref(q, k, v, causal: bool, scale: float,
             g = kv_head_of(h, Hq, Hkv)
             for i0 in range(0, N, block_q):
                 rows = np.arange(i0, min(N, i0 + block_q))
-                Qb = q[b, h, rows]
-                O = np.zeros((len(rows), d))
-                m = np.full(len(rows), -np.inf)
-                l = np.zeros(len(rows))
-                for j0 in range(0, N, block_k):
-                    cols = np.arange(j0, min(N, j0 + block_k))
-                    S = scale * (Qb @ k[b, g, cols].T)
+                state = (np.full(len(rows), -np.inf), np.zeros(len(rows)), np.zeros((len(rows), d)))
+                for jb in order:
+                    cols = np.arange(starts[jb], min(N, starts[jb] + block_k))
+                    S = scale * (q[b, h, rows] @ k[b, g, cols].T)
                     if _masked(causal, window, prefix):
                         S[~visible(rows, cols, True, window, prefix)] = -np.inf
-                    m_new = np.maximum(m, S.max(axis=1))
-                    # A row whose blocks so far are all masked keeps m = -inf;
-                    # its factors are then defined as 1 (nothing to rescale).
-                    safe = np.where(np.isneginf(m_new), 0.0, m_new)
-                    alpha = np.where(np.isneginf(m_new), 1.0, np.exp(m - safe))
-                    E = np.exp(S - safe[:, None])
-                    l = alpha * l + E.sum(axis=1)
-                    O = alpha[:, None] * O + E @ v[b, g, cols]
-                    m = m_new
-                O_out[b, h, rows] = O / l[:, None]
+                    state = merge_softmax_states(state, softmax_state(S, v[b, g, cols]))
+                m, l, U = state
+                O_out[b, h, rows] = U / l[:, None]
                 L_out[b, h, rows] = m + np.log(l)
     return O_out, L_out
 

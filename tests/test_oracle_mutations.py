@@ -73,6 +73,49 @@ def test_forward_mutation_is_caught(monkeypatch, name, target, repl):
     assert _fails(FWD_CHECKS), name
 
 
+_orig_merge = A.merge_softmax_states
+
+
+def merge_second_not_rescaled(a, b):
+    # Forgets to bring the second state to the common maximum.
+    ma, la, Ua = a
+    mb, lb, Ub = b
+    M = np.maximum(ma, mb)
+    ref = np.where(np.isneginf(M), 0.0, M)
+    fa = np.where(np.isneginf(ma), 0.0, np.exp(ma - ref))
+    fb = np.where(np.isneginf(mb), 0.0, 1.0)
+    return M, fa * la + fb * lb, fa[:, None] * Ua + fb[:, None] * Ub
+
+
+def merge_output_not_rescaled(a, b):
+    # Rescales the sums but not the partial outputs.
+    M, l, _ = _orig_merge(a, b)
+    return M, l, a[2] + b[2]
+
+
+def merge_sign_flipped(a, b):
+    # e^(M - m) instead of e^(m - M).
+    ma, la, Ua = a
+    mb, lb, Ub = b
+    M = np.maximum(ma, mb)
+    ref = np.where(np.isneginf(M), 0.0, M)
+    fa = np.where(np.isneginf(ma), 0.0, np.exp(ref - ma))
+    fb = np.where(np.isneginf(mb), 0.0, np.exp(ref - mb))
+    return M, fa * la + fb * lb, fa[:, None] * Ua + fb[:, None] * Ub
+
+
+@pytest.mark.parametrize("name,repl", [
+    ("second state not rescaled", merge_second_not_rescaled),
+    ("partial outputs not rescaled", merge_output_not_rescaled),
+    ("rescale exponent sign flipped", merge_sign_flipped),
+])
+def test_merge_mutation_is_caught(monkeypatch, name, repl):
+    monkeypatch.setattr(A, "merge_softmax_states", repl)
+    monkeypatch.setattr(oracle, "merge_softmax_states", repl)
+    assert _fails([pins.check_online_equals_two_pass, pins.check_online_any_merge_order,
+                   pins.check_merge_closed_form]), name
+
+
 def _wrap_bwd(kind):
     ref = oracle.attn_bwd_ref
 

@@ -97,6 +97,67 @@ def test_online_equals_two_pass():
     check_online_equals_two_pass()
 
 
+def check_online_any_merge_order():
+    # The merge of partial softmax states is associative and commutative, so
+    # merging the key blocks in any order gives the two-pass result.
+    rng = np.random.default_rng(71)
+    for causal, N, bk in [(False, 37, 5), (True, 37, 5), (True, 64, 16), (False, 9, 1)]:
+        q = rnd((1, 2, N, 6), 71 + N, 2.0)
+        k = rnd((1, 1, N, 6), 72 + N, 2.0)
+        v = rnd((1, 1, N, 6), 73 + N)
+        O, L = oracle.attn_fwd_ref(q, k, v, causal, 0.7)
+        nb = (N + bk - 1) // bk
+        for order in [list(range(nb))[::-1], list(rng.permutation(nb)), list(rng.permutation(nb))]:
+            Oo, Lo = oracle.attn_fwd_online_ref(q, k, v, causal, 0.7, 7, bk, order=order)
+            np.testing.assert_allclose(Oo, O, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(Lo, L, rtol=1e-12, atol=1e-12)
+
+
+def test_online_any_merge_order():
+    check_online_any_merge_order()
+
+
+def check_merge_closed_form():
+    # Two keys with scores s1, s2 and values v1, v2, one per block: the merged
+    # state must give softmax weights e^s / (e^s1 + e^s2) and L = ln(e^s1 + e^s2),
+    # computed here with math.exp / math.fsum.
+    for s1, s2 in [(0.3, -1.2), (5.0, 5.0), (-40.0, 2.5), (700.0, 699.0)]:
+        v1, v2 = np.array([1.0, -2.0, 0.5]), np.array([3.0, 0.25, -1.0])
+        a = oracle.softmax_state(np.array([[s1]]), v1[None])
+        b = oracle.softmax_state(np.array([[s2]]), v2[None])
+        mx = max(s1, s2)
+        e1, e2 = math.exp(s1 - mx), math.exp(s2 - mx)
+        want_o = (e1 * v1 + e2 * v2) / math.fsum([e1, e2])
+        want_l = mx + math.log(math.fsum([e1, e2]))
+        for m, l, U in (oracle.merge_softmax_states(a, b), oracle.merge_softmax_states(b, a)):
+            np.testing.assert_allclose(U[0] / l[0], want_o, rtol=1e-14, atol=1e-14)
+            assert abs(m[0] + math.log(l[0]) - want_l) <= 1e-12 * max(1.0, abs(want_l))
+    # The empty state (every key of a block masked) is the identity, exactly.
+    empty = oracle.softmax_state(np.full((1, 4), -np.inf), np.ones((4, 3)))
+    assert np.isneginf(empty[0]).all() and (empty[1] == 0).all() and (empty[2] == 0).all()
+    a = oracle.softmax_state(np.array([[0.5, -0.25]]), np.array([[1.0, 2.0, 3.0], [4.0, 5.0, 6.0]]))
+    for merged in (oracle.merge_softmax_states(a, empty), oracle.merge_softmax_states(empty, a)):
+        for x, y in zip(merged, a):
+            assert np.array_equal(x, y)
+
+
+def test_merge_closed_form():
+    check_merge_closed_form()
+
+
+def test_online_matches_brute_force():
+    # The blocked online form against pure-Python loops (independent of the
+    # two-pass oracle), causal and not, blocks that do not divide N.
+    for causal in (False, True):
+        q = rnd((1, 2, 7, 3), 91, 1.5)
+        k = rnd((1, 1, 7, 3), 92, 1.5)
+        v = rnd((1, 1, 7, 3), 93)
+        O, L = brute_fwd(q, k, v, causal, 0.8)
+        Oo, Lo = oracle.attn_fwd_online_ref(q, k, v, causal, 0.8, 3, 2)
+        np.testing.assert_allclose(Oo, O, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(Lo, L, rtol=1e-13, atol=1e-13)
+
+
 def check_rows_sum_to_one(fwd=None):
     # A V column of ones returns sum_j P_ij, which must be 1 in every row.
     fwd = fwd or oracle.attn_fwd_ref
