@@ -107,30 +107,30 @@ def load_peaks():
 
 
 def captured_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch of ``kernel`` on ``workload`` from the ncu table
-    in profiles/traffic.md, or None when there is no row or the kernel's
-    sources changed since the capture (sha256 of their concatenation)."""
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from the ncu
+    capture table profiles/traffic.json, or None when there is no entry or
+    the kernel's sources changed since the capture (sha256 of their
+    concatenation, first 16 hex digits)."""
     import hashlib
 
     try:
-        with open(os.path.join(ROOT, "profiles", "traffic.md")) as f:
-            lines = f.read().splitlines()
-    except OSError:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            captures = json.load(f)["captures"]
+    except (OSError, ValueError, KeyError):
         return None
-    for ln in lines:
-        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
-        if len(cells) != 5 or cells[0] != kernel or cells[1] != workload:
+    for c in captures:
+        if c.get("kernel") != kernel or c.get("workload") != workload:
             continue
         m = hashlib.sha256()
         try:
-            for src in cells[2].split():
+            for src in c["sources"]:
                 with open(os.path.join(ROOT, "exact_io_aware_56_b200", "csrc", src), "rb") as f:
                     m.update(f.read())
-        except OSError:
+        except (OSError, KeyError):
             return None
-        if m.hexdigest()[:16] != cells[3]:
+        if m.hexdigest()[:16] != c.get("sha256_16"):
             return None
-        return int(cells[4])
+        return int(c["traffic_bytes"])
     return None
 
 
@@ -157,13 +157,18 @@ class ClockSampler:
         self._thread = None
         self._proc = None
 
-    def _nvml_handle(self):
-        import pynvml
+    def _bus_id(self):
+        """PCI bus id of the CUDA device (unaffected by CUDA_VISIBLE_DEVICES)."""
         import torch
 
-        pynvml.nvmlInit()
         p = torch.cuda.get_device_properties(self.device)
-        bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        bus = self._bus_id()
         for arg in (bus, bus.encode()):
             try:
                 return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(arg)
@@ -203,13 +208,21 @@ class ClockSampler:
             self._thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h), daemon=True)
         except Exception as exc:
             print(f"bench.py: NVML clock sampling unavailable ({exc}); using nvidia-smi", file=sys.stderr)
+            # nvidia-smi numbers GPUs physically; the torch index is not that
+            # number under CUDA_VISIBLE_DEVICES, the PCI bus id always is.
             try:
-                self._proc = subprocess.Popen(
-                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
-                     "-i", str(self.device.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-                self._thread = threading.Thread(target=self._poll_smi, daemon=True)
-            except OSError:
-                self._thread = None
+                target = self._bus_id()
+            except Exception:
+                target = None if "CUDA_VISIBLE_DEVICES" in os.environ else str(self.device.index)
+            self._thread = None
+            if target is not None:
+                try:
+                    self._proc = subprocess.Popen(
+                        ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                         "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                    self._thread = threading.Thread(target=self._poll_smi, daemon=True)
+                except OSError:
+                    self._thread = None
         if self._thread is not None:
             self._thread.start()
         return self

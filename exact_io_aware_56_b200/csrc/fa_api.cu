@@ -121,6 +121,13 @@ LaunchCtl make_ctl(const DevState* st) {
 
 }  // namespace
 
+int check_current_device() {
+  DevState* st = nullptr;
+  return device_state(&st);
+}
+
+int record_cuda_error(cudaError_t e) { return record_cuda(e); }
+
 namespace {
 bool encode_map(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, int cols, int rows,
                 int outer, int box_cols, int box_rows) {

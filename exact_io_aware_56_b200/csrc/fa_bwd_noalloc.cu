@@ -30,12 +30,10 @@ constexpr int kMaxDevices = 64;
 // device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_bwd_scratch[kScratchBytes];
 
-struct ScratchAddr {
-  std::once_flag once;
-  cudaError_t status = cudaErrorUnknown;
-  void* ptr = nullptr;
-};
-ScratchAddr g_addr[kMaxDevices];
+// Device address of the array per device. Only a successful lookup is
+// kept; a failed one is retried by the next call.
+std::mutex g_addr_mu;
+void* g_addr[kMaxDevices] = {};
 
 }  // namespace
 
@@ -49,12 +47,28 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
     return (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0) ? FA_ERR_INVALID_ARGUMENT : FA_ERR_UNSUPPORTED;
   }
   if (need > kScratchBytes) return FA_ERR_UNSUPPORTED;
+  // The device check of every entry point comes first, so that a device
+  // this library has no kernels for reports FA_ERR_UNSUPPORTED.
+  int rc = fa::check_current_device();
+  if (rc != FA_OK) return rc;
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fa::record_cuda_error(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
   // Set-up, once per device, with that device current: the device address
   // of the array.
-  ScratchAddr& a = g_addr[dev];
-  std::call_once(a.once, [&] { a.status = cudaGetSymbolAddress(&a.ptr, g_bwd_scratch); });
-  if (a.status != cudaSuccess || a.ptr == nullptr) return FA_ERR_CUDA;
-  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, a.ptr, kScratchBytes, stream);
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_addr_mu);
+    if (g_addr[dev] == nullptr) {
+      e = cudaGetSymbolAddress(&ptr, g_bwd_scratch);
+      if (e != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();  // clear the last-error state; the next call retries the lookup
+        return fa::record_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      }
+      g_addr[dev] = ptr;
+    }
+    ptr = g_addr[dev];
+  }
+  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, ptr, kScratchBytes, stream);
 }

@@ -47,6 +47,15 @@ bool encode_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int
 bool encode_f32_tile_map(CUtensorMap* map, const void* base, int cols, int rows, int outer, int box_cols,
                          int box_rows);
 
+// Checks that the current device is supported (compute capability 10.0),
+// once per device, as every entry point does before its first launch.
+// Returns FA_OK or the entry points' error status.
+int check_current_device();
+
+// Keeps `e` as the message of FA_ERR_CUDA for fa_status_string and returns
+// FA_ERR_CUDA.
+int record_cuda_error(cudaError_t e);
+
 // o_resid may be null (no residual written).
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream);

@@ -116,9 +116,9 @@ def test_captured_traffic_requires_unchanged_sources(tmp_path, monkeypatch):
     (csrc / "k.cu").write_bytes(b"kernel source v1")
     digest = hashlib.sha256(b"kernel source v1").hexdigest()[:16]
     (tmp_path / "profiles").mkdir()
-    (tmp_path / "profiles" / "traffic.md").write_text(
-        "| kernel | workload | sources | sha256/16 | traffic bytes |\n|---|---|---|---|---|\n"
-        f"| kern | wl | k.cu | {digest} | 12345 |\n")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"captures": [{"kernel": "kern", "workload": "wl", "sources": ["k.cu"], "sha256_16": digest,
+                       "traffic_bytes": 12345}]}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.captured_traffic("kern", "wl") == 12345
     assert bench.captured_traffic("kern", "other") is None

@@ -1,5 +1,6 @@
-"""The convenience calls shown in the README, at a smaller N, checked
-against the oracle (so that the documented usage keeps working)."""
+"""The convenience calls of the Python binding (attention_forward,
+attention_backward, attention_decode, attention_forward_fp8) used the way a
+caller would, at a smaller N, checked against the oracle."""
 
 import numpy as np
 import pytest

@@ -2,17 +2,19 @@
 memory (hosts that pass a library only its inputs and outputs, or that
 forbid cudaMalloc). Its workspace is a fixed device array inside libfa. This
 test calls it through the C ABI twice in a row and checks each result
-against the existing fa_bwd entry point given a caller-owned workspace.
+element by element against the fp64 oracle (attn_bwd_ref) and against the
+existing fa_bwd entry point given a caller-owned workspace, both within the
+tolerance of the other GPU parity tests.
 
 The file name makes pytest collect it after every other test file.
 """
 
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
+import oracle
 from exact_io_aware_56_b200 import fa, make_inputs, to_f64
 
 from .parity import assert_close_abs
@@ -31,16 +33,18 @@ def _noalloc():
     return f
 
 
-def test_noalloc_matches_fa_bwd_twice():
+def test_noalloc_matches_oracle_and_fa_bwd_twice():
     B, Hq, Hkv, N, d, causal = 1, 4, 2, 1000, 128, True
     assert fa.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) <= SCRATCH_BYTES
     scale = d ** -0.5
     host = make_inputs(B, Hq, Hkv, N, d, seed=2024)
     dev = {k: v.cuda() for k, v in host.items()}
+    ref = {k: to_f64(v) for k, v in host.items()}
+    want = oracle.attn_bwd_ref(ref["q"], ref["k"], ref["v"], ref["dout"], causal, scale)
     o, lse = fa.attention_forward(dev["q"], dev["k"], dev["v"], causal, scale)
-    ref = fa.attention_backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, causal, scale)
+    lib_out = fa.attention_backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, causal, scale)
     torch.cuda.synchronize()
-    ref = [to_f64(t) for t in ref]
+    lib_out = [to_f64(t) for t in lib_out]
     f = _noalloc()
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
@@ -51,8 +55,9 @@ def test_noalloc_matches_fa_bwd_twice():
         assert rc == fa.FA_OK, fa.status_string(rc)
         torch.cuda.synchronize()
         assert fa.fa_check_device_error() == fa.FA_OK
-        for name, got, want in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
-            assert_close_abs(f"{name} (call {call + 1})", to_f64(got), want)
+        for name, got, w, lo in zip(("dQ", "dK", "dV"), (dq, dk, dv), want, lib_out):
+            assert_close_abs(f"{name} vs oracle (call {call + 1})", to_f64(got), w)
+            assert_close_abs(f"{name} vs fa_bwd (call {call + 1})", to_f64(got), lo)
 
 
 def test_noalloc_rejects_shapes_beyond_its_array():
