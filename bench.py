@@ -42,6 +42,8 @@ METRIC = "attention fwd/bwd TFLOP/s (bf16) and fraction of B200 dense BF16 peak"
 FP8_METRIC = "attention forward TFLOP/s in FP8 mode (e4m3 operands, block scales) and fraction of B200 dense FP8 peak"
 DECODE_METRIC = "decode attention: algorithmic HBM bytes per second (read q, K/V cache; write o, lse)"
 DEFAULT_WORKLOAD = "fwdbwd_b2_h16_n8192_d128_causal_peaky"
+L2_BYTES = 126 << 20     # B200 L2
+FLUSH_BYTES = 512 << 20  # written before each timed step when the inputs do not exceed 2x L2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -315,21 +317,52 @@ def pipelined_e2e(dev, compute_stream, host_in, make_set, run, steps):
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample(w, seconds: float, max_slices: int = 64):
-    """Times the fp64 oracle (as it stands) on whole (batch, head) slices of
-    the workload until about ``seconds`` have passed. Returns
-    (algorithmic FLOPs done, wall seconds, slices, threads)."""
-    import oracle
-    from exact_io_aware_56_b200 import make_inputs, to_f64
+# A (batch, head) slice whose forward costs more than this many algorithmic
+# FLOPs is sampled by query rows instead of whole (the 131072-token forward:
+# ~4.4 TFLOP per slice, hours of fp64 work).
+ROW_SAMPLE_ABOVE_FLOPS = 200e9
 
+
+def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
 
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # pragma: no cover - threadpoolctl missing
-        threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+        return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def oracle_sample(w, seconds: float, max_slices: int = 64):
+    """Times the fp64 oracle (as it stands) on whole (batch, head) slices of
+    the workload until about ``seconds`` have passed. Returns
+    (algorithmic FLOPs done, wall seconds, units done, threads, unit name).
+
+    A forward-only workload whose slice is too large for that (more than
+    ROW_SAMPLE_ABOVE_FLOPS) is timed on chunks of 64 seeded query rows of
+    one slice instead (``attn_fwd_rows``), each row counted at its
+    algorithmic cost 4 * (visible keys) * d."""
+    import numpy as np
+
+    import oracle
+    from exact_io_aware_56_b200 import make_inputs, sample_rows, to_f64
+
+    threads = _blas_threads()
     flops_slice = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.Hq)
     done, elapsed, n = 0.0, 0.0, 0
+    if not w.backward and w.fwd_flops() / (w.B * w.Hq) > ROW_SAMPLE_ABOVE_FLOPS:
+        host = make_inputs(1, 1, 1, w.N, w.d, w.seed + 7919, w.qk_gain, False)
+        ref = {k: to_f64(v) for k, v in host.items()}
+        order = sample_rows(w.N, min(w.N, 64 * 4096), w.seed + 7919)
+        np.random.default_rng(w.seed).shuffle(order)
+        while n < max_slices * 64 and (elapsed < seconds or n == 0):
+            rows = np.sort(order[n * 64:(n + 1) * 64])
+            t0 = time.perf_counter()
+            oracle.attn_fwd_rows(ref["q"], ref["k"], ref["v"], w.causal, w.scale, 0, 0, rows)
+            elapsed += time.perf_counter() - t0
+            keys = (rows + 1) if w.causal else np.full(len(rows), w.N)
+            done += float(4.0 * keys.sum() * w.d)
+            n += 1
+        return done, elapsed, n, threads, "chunks of 64 query rows of one (batch, head) slice"
     while n < max_slices and (elapsed < seconds or n == 0):
         host = make_inputs(1, 1, 1, w.N, w.d, w.seed + 7919 * (n + 1), w.qk_gain, w.backward)
         ref = {k: to_f64(v) for k, v in host.items()}
@@ -340,7 +373,7 @@ def oracle_sample(w, seconds: float, max_slices: int = 64):
         elapsed += time.perf_counter() - t0
         done += flops_slice
         n += 1
-    return done, elapsed, n, threads
+    return done, elapsed, n, threads, "whole (batch, head) slices"
 
 
 def decode_oracle_sample(w, seconds: float, max_batches: int = 64):
@@ -350,12 +383,7 @@ def decode_oracle_sample(w, seconds: float, max_batches: int = 64):
     import oracle
     from exact_io_aware_56_b200 import make_decode_inputs, to_f64
 
-    try:
-        from threadpoolctl import threadpool_info
-
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # pragma: no cover - threadpoolctl missing
-        threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    threads = _blas_threads()
     bytes_batch = w.bytes_moved() / w.B
     done, elapsed, n = 0.0, 0.0, 0
     while n < max_batches and (elapsed < seconds or n == 0):
@@ -406,12 +434,7 @@ def fp8_oracle_sample(w, seconds: float, max_slices: int = 64):
     import oracle
     from exact_io_aware_56_b200 import make_inputs, to_f64
 
-    try:
-        from threadpoolctl import threadpool_info
-
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # pragma: no cover - threadpoolctl missing
-        threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    threads = _blas_threads()
     flops_slice = w.fwd_flops() / (w.B * w.Hq)
     done, elapsed, n = 0.0, 0.0, 0
     while n < max_slices and (elapsed < seconds or n == 0):
@@ -465,16 +488,17 @@ def reference_arm(args):
     if rank != 0:
         return 0
     w = WORKLOADS[args.workload]
-    times = []
-    flops_slice = (w.fwd_flops() + w.bwd_flops()) / (w.B * w.Hq)
-    threads = 1
+    times, flops = [], []
+    threads, unit = 1, ""
     for it in range(args.warmup + args.steps):
-        _, el, _, threads = oracle_sample(w, 0.0, max_slices=1)
+        f, el, _, threads, unit = oracle_sample(w, 0.0, max_slices=1)
         if it >= args.warmup:
             times.append(el)
+            flops.append(f)
     ms = 1e3 * sum(times) / len(times)
-    value = flops_slice / (ms * 1e-3) / 1e12
-    sample = f"one (batch, head) slice of {w.name} (fwd+bwd, fp64 oracle) per step"
+    value = sum(flops) / (sum(times) or 1e-30) / 1e12
+    passes = "fwd+bwd" if w.backward else "fwd"
+    sample = f"one of the {unit} of {w.name} ({passes}, fp64 oracle) per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -539,6 +563,12 @@ def native_arm(args):
     for e in evs:  # torch creates the CUDA event on first record; the hook needs real handles
         e[2].record(stream)
         e[3].record(stream)
+    # Inputs smaller than twice L2: L2 is flushed (a buffer larger than L2
+    # is written) before every timed step, outside its events, and the time
+    # is the sum of the steps' own event intervals.
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v) + ((dout,) if w.backward else ()))
+    flush = in_bytes < 2 * L2_BYTES
+    scratch = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize(dev)
@@ -547,6 +577,8 @@ def native_arm(args):
         clocks.begin()
         t_start.record(stream)
         for s in range(args.steps):
+            if flush:
+                scratch.fill_(s & 0xFF)
             if w.backward:
                 fa.fa_profile_set_bwd_events(evs[s][2], evs[s][3])
             step(evs[s])
@@ -557,7 +589,7 @@ def native_arm(args):
     barrier(dev)
     if fa.fa_check_device_error(stream) != fa.FA_OK:
         raise RuntimeError("device watchdog fired during the timed steps")
-    ms_local = t_start.elapsed_time(t_end)
+    ms_local = sum(e[0].elapsed_time(e[4]) for e in evs) if flush else t_start.elapsed_time(t_end)
     ms_total = max_over_ranks(ms_local, dev)
     step_flops = w.fwd_flops() + w.bwd_flops()
     value = step_flops * args.steps * world / (ms_total * 1e-3) / 1e12
@@ -620,11 +652,14 @@ def native_arm(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        flops, secs, n, threads = oracle_sample(w, args.cpu_seconds)
+        flops, secs, n, threads, unit = oracle_sample(w, args.cpu_seconds)
+        passes = "fwd+bwd" if w.backward else "fwd"
         cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n} whole (batch, head) slices of {w.name}, fwd+bwd, fp64 oracle, {secs:.1f} s"}
+               "sample": f"{n} {unit} of {w.name}, {passes}, fp64 oracle, {secs:.1f} s"}
 
-    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v) + ((dout,) if w.backward else ()))
+    l2_note = (f"inputs {in_bytes / 2**20:.0f} MiB per rank, L2 flushed before every step "
+               f"({FLUSH_BYTES >> 20} MiB write, outside the step's events)" if flush else
+               f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per rank), no flush")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
@@ -632,7 +667,7 @@ def native_arm(args):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                    "causal": w.causal, "qk_gain": w.qk_gain, "global_batch": w.B * world,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB per rank), no flush"},
+                   "l2": l2_note},
         "fraction_of_peak": value / world / peak,
         "roofline": roofline,
         "cpu_baseline": cpu,

@@ -24,7 +24,7 @@
 //               P^T  = 2^(S^T scale log2e - L_i log2e), dS^T = P^T o (dP^T - D_i)
 //                                         (one thread per key row)
 //               dV_j += P^T dO_i          (P^T read from tensor memory)
-//               dK_j += dS^T Q_i          (dS^T from shared memory)
+//               dK_j += dS^T Q_i          (dS^T read from tensor memory)
 //               dQ_i^T = K_j^T dS_i^T     (M = d: one thread per column of dQ)
 //             dQ_i is added to the fp32 accumulator by coalesced reductions
 //             issued from registers, which overlap the next tiles.
@@ -34,27 +34,33 @@
 // Warp roles of bwd_main (512 threads):
 //   warps 0-3   softmax-gradient warpgroup for even query tiles (buffer 0),
 //   warps 4-7   the same for odd tiles (buffer 1): thread = key row; writes
-//               P^T to tensor memory and dS^T to shared memory; epilogue
-//               stores dV (half of the columns each).
+//               P^T and dS^T to tensor memory and dS^T to shared memory (the
+//               B operand of dQ^T); epilogue stores dV (half of the columns
+//               each).
 //   warp 8      producer: K_j, V_j once; Q_i, dO_i by TMA and L_i, D_i by
 //               plain loads into a three-stage ring.
-//   warp 9      tensor-memory owner and MMA issuer.
+//   warp 9      tensor-memory owner and MMA issuer (the whole warp runs the
+//               issue loop so operand descriptors stay warp-uniform; one
+//               elected lane issues).
 //   warps 10-11 idle (keep the third warpgroup whole).
 //   warps 12-15 dQ warpgroup: thread = column c of dQ; reads dQ_i^T out of
 //               tensor memory, releases it and issues the reductions;
 //               epilogue stores dK.
-// Tensor memory (512 columns): S^T[2] (64 each) | dP^T[2] (64 each; P^T in
-// bf16 over its first 32 columns, then dQ_i^T over all 64) | dV (D) | dK (D).
+// Tensor memory (512 columns): S^T[2] (64 each; dS^T in bf16 over its first
+// 32 columns once S^T is loaded) | dP^T[2] (64 each; P^T in bf16 over its
+// first 32 columns, then dQ_i^T over all 64) | dV (D) | dK (D).
 // S^T and dP^T are double-buffered so that one warpgroup's softmax-gradient
 // work overlaps the MMAs of the other's tile. Every tcgen05 operation of the
 // MMA thread completes in issue order, which orders the P^T reads of dV
-// before the dQ^T write into the same columns.
+// before the dQ^T write into the same columns, and the dS^T reads of dK
+// before the next S^T write into its columns.
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include "fa_internal.h"
 #include "sm100.cuh"
+
 
 namespace fa {
 namespace {
@@ -98,6 +104,7 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   int N, Hq, Hkv, BHkv, nk, nq;
   int group;  // KV heads per scheduling group (see the work-unit comment)
+  int band;   // causal: key tiles per scheduling band (0: strict longest-first)
   int window;  // left window (a huge value when there is none), mask kind 2
   int prefix;  // prefix length, mask kind 2
   float scale, scale_log2;
@@ -150,12 +157,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   // otherwise small enough that their query heads' Q, dO and dQ-accumulator
   // tiles stay in L2 while the resident CTAs sweep them); within a group the
   // longest units (smallest j when causal) come first.
-  const int per_group = a.group * a.nk;
-  const int grp = blockIdx.x / per_group;
-  const int rem = blockIdx.x - grp * per_group;
-  const int gsize = min(a.group, a.BHkv - grp * a.group);
-  const int bkv = grp * a.group + rem % gsize;
-  const int j = rem / gsize;
+  int bkv, j;
+  if (MASK == 1 && a.band > 0) {
+    // Bands of a.band key tiles, longest band first; within a band,
+    // KV-head-major with the key tiles of a head adjacent, so that the
+    // resident CTAs share the dQ accumulator, Q and dO of a few heads.
+    const int per_band = a.band * a.BHkv;
+    const int band = blockIdx.x / per_band;
+    const int rem = blockIdx.x - band * per_band;
+    const int bw = min(a.band, a.nk - band * a.band);
+    bkv = rem / bw;
+    j = band * a.band + rem % bw;
+  } else {
+    const int per_group = a.group * a.nk;
+    const int grp = blockIdx.x / per_group;
+    const int rem = blockIdx.x - grp * per_group;
+    const int gsize = min(a.group, a.BHkv - grp * a.group);
+    bkv = grp * a.group + rem % gsize;
+    j = rem / gsize;
+  }
   const int r = a.Hq / a.Hkv;
   const int b = bkv / a.Hkv;
   const int g = bkv % a.Hkv;
@@ -268,75 +288,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
+    // The whole warp runs this loop (descriptors stay warp-uniform); the
+    // elected lane issues the tcgen05 instructions.
+    const bool leader = elect_one();
+    auto all = [](bool b) { return __all_sync(0xffffffffu, b); };
+    {
       constexpr uint32_t id_sdp = idesc_bf16(kKT, kQT, false, false);  // S^T, dP^T: 128 x 64
       constexpr uint32_t id_dvk = idesc_bf16(kKT, D, false, true);     // dV (A in TMEM), dK
       constexpr uint32_t id_dq = idesc_bf16(128, kQT, true, true);     // dQ^T: A = K^T, B = dS^T
-      // K-major operand of a 128-row tile (64-column boxes kKBox apart).
-      auto kdesc_k = [](uint32_t base, int k) {
-        return sdesc_sw128(base + (k / 4) * (kKT * 128) + (k % 4) * 32, 16, 1024);
+      // Operand descriptors, computed once and stepped by byte offsets
+      // (sdesc_step). K step k (16 elements) of a K-major operand: 32 bytes
+      // within a 128-byte swizzle row, boxes of 64 columns kKBox / kQBox
+      // bytes apart; of an MN-major operand: 16 rows of 128 bytes (2048).
+      const uint64_t kK = sdesc_sw128(sK, 16, 1024), kV = sdesc_sw128(sV, 16, 1024);
+      const uint64_t kQ = sdesc_sw128(sQ, 16, 1024), kO = sdesc_sw128(sDO, 16, 1024);
+      const uint64_t kDS = sdesc_sw128(sDS, 16, 1024);
+      const uint64_t mQ = sdesc_sw128(sQ, C::kQBox, 1024), mO = sdesc_sw128(sDO, C::kQBox, 1024);
+      const uint64_t mK = sdesc_sw128(sK, C::kKBox, 1024), mDS = sdesc_sw128(sDS, C::kKBox, 1024);
+      auto ofs_k = [](int k) { return static_cast<uint32_t>((k / 4) * (kKT * 128) + (k % 4) * 32); };
+      auto ofs_q = [](int k) { return static_cast<uint32_t>((k / 4) * (kQT * 128) + (k % 4) * 32); };
+      auto ofs_m = [](int k) { return static_cast<uint32_t>(k * 2048); };
+      // Four MMAs, K steps k0..k0+3, into d; A and B stepped by their offsets.
+      auto ss4 = [&](uint32_t d, uint64_t a, uint64_t b, auto oa, auto ob, int k0, uint32_t id, uint32_t acc0) {
+        mma_ss_x4(d, sdesc_step(a, oa(k0)), sdesc_step(a, oa(k0 + 1)), sdesc_step(a, oa(k0 + 2)),
+                  sdesc_step(a, oa(k0 + 3)), sdesc_step(b, ob(k0)), sdesc_step(b, ob(k0 + 1)),
+                  sdesc_step(b, ob(k0 + 2)), sdesc_step(b, ob(k0 + 3)), id, acc0, leader);
       };
-      // K-major operand of a 64-row tile.
-      auto kdesc_q = [](uint32_t base, int k) {
-        return sdesc_sw128(base + (k / 4) * (kQT * 128) + (k % 4) * 32, 16, 1024);
+      auto ts4 = [&](uint32_t d, uint32_t a, uint64_t b, auto ob, int k0, uint32_t id, uint32_t acc0) {
+        mma_ts_x4(d, a + 8 * k0, a + 8 * (k0 + 1), a + 8 * (k0 + 2), a + 8 * (k0 + 3), sdesc_step(b, ob(k0)),
+                  sdesc_step(b, ob(k0 + 1)), sdesc_step(b, ob(k0 + 2)), sdesc_step(b, ob(k0 + 3)), id, acc0,
+                  leader);
       };
-      // MN-major operands, K step k (16 rows): 64-column chunks `lbo` apart.
-      auto mdesc = [](uint32_t base, int k, uint32_t lbo) { return sdesc_sw128(base + k * 2048, lbo, 1024); };
       auto issue_sdp = [&](int it) {
         const int x = it & 1;
-        const uint32_t q = sQ + (it % kQStages) * C::kQTile, o = sDO + (it % kQStages) * C::kQTile;
+        const uint32_t st = (it % kQStages) * C::kQTile;
+        const uint64_t q = sdesc_step(kQ, st), o = sdesc_step(kO, st);
         const uint32_t tS = tmem + C::kColS + 64 * x, tDP = tmem + C::kColDP + 64 * x;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) mma_ss(tS, kdesc_k(sK, k), kdesc_q(q, k), id_sdp, k > 0);
-        mma_commit(&bars->s_full[x]);
+        for (int k = 0; k < D / 16; k += 4) ss4(tS, kK, q, ofs_k, ofs_q, k, id_sdp, k > 0);
+        mma_commit(&bars->s_full[x], leader);
         return [=] {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) mma_ss(tDP, kdesc_k(sV, k), kdesc_q(o, k), id_sdp, k > 0);
+          for (int k = 0; k < D / 16; k += 4) ss4(tDP, kV, o, ofs_k, ofs_q, k, id_sdp, k > 0);
         };
       };
       const uint32_t tDV = tmem + C::kColDV, tDK = tmem + C::kColDK;
-      bool ok = wait_bar(&bars->kv_full, 0, w);
+      // M(it): dV += P^T dO, dK += dS^T Q, dQ^T = K^T dS^T for tile it.
+      auto issue_main = [&](int it) {
+        const int x = it & 1;
+        const int s = it % kQStages;
+        const uint32_t tDP = tmem + C::kColDP + 64 * x;
+        const uint32_t st = s * C::kQTile;
+        const uint64_t qm = sdesc_step(mQ, st), om = sdesc_step(mO, st);
+        const uint32_t acc = it > 0;
+        ts4(tDV, tDP, om, ofs_m, 0, id_dvk, acc);  // dV += P^T dO (K = 64 queries)
+        ts4(tDK, tmem + C::kColS + 64 * x, qm, ofs_m, 0, id_dvk, acc);  // dK += dS^T Q (dS^T in tensor memory)
+        const uint64_t dsm = sdesc_step(mDS, x * C::kDSTile);
+#pragma unroll
+        for (int k = 0; k < kKT / 16; k += 4) ss4(tDP, mK, dsm, ofs_m, ofs_m, k, id_dq, k > 0);  // dQ^T = K^T dS^T
+        mma_commit(&bars->dq_full[x], leader);
+        mma_commit(&bars->ds_free[x], leader);
+        mma_commit(&bars->q_empty[s], leader);
+      };
+      bool ok = all(wait_bar(&bars->kv_full, 0, w));
+      // Tiles 0 and 1: S^T and dP^T into their own buffers.
       for (int it = 0; ok && it < 2 && it < n_it; ++it) {
-        if (!(ok = wait_bar(&bars->q_full[it % kQStages], (it / kQStages) & 1, w))) break;
+        if (!(ok = all(wait_bar(&bars->q_full[it % kQStages], (it / kQStages) & 1, w)))) break;
         tc_fence_after();
         auto dp = issue_sdp(it);
         dp();
-        mma_commit(&bars->dp_full[it & 1]);
+        mma_commit(&bars->dp_full[it & 1], leader);
       }
+      // Then, per tile it: M(it) once the softmax-gradient warps hand it
+      // back; S^T and dP^T of tile it + 2 into the same buffers (dP^T after
+      // dQ^T of tile it has been read out of its columns).
       for (int it = 0; ok && it < n_it; ++it) {
         const int x = it & 1;
-        const int s = it % kQStages;
-        const uint32_t q = sQ + s * C::kQTile, o = sDO + s * C::kQTile;
-        const uint32_t tDP = tmem + C::kColDP + 64 * x;
-        const uint32_t ds = sDS + x * C::kDSTile;
-        if (!(ok = wait_bar(&bars->p_ready[x], (it >> 1) & 1, w))) break;
+        if (!(ok = all(wait_bar(&bars->p_ready[x], (it >> 1) & 1, w)))) break;
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kQT / 16; ++k)  // dV += P^T dO (K = 64 queries)
-          mma_ts(tDV, tDP + 8 * k, mdesc(o, k, C::kQBox), id_dvk, (it > 0 || k > 0));
-#pragma unroll
-        for (int k = 0; k < kQT / 16; ++k)  // dK += dS^T Q
-          mma_ss(tDK, kdesc_q(ds, k), mdesc(q, k, C::kQBox), id_dvk, (it > 0 || k > 0));
-#pragma unroll
-        for (int k = 0; k < kKT / 16; ++k)  // dQ^T = K^T dS^T (K = 128 keys)
-          mma_ss(tDP, mdesc(sK, k, C::kKBox), mdesc(ds, k, C::kKBox), id_dq, k > 0);
-        mma_commit(&bars->dq_full[x]);
-        mma_commit(&bars->ds_free[x]);
-        mma_commit(&bars->q_empty[s]);
+        issue_main(it);
         const int nx = it + 2;
         if (nx < n_it) {
-          if (!(ok = wait_bar(&bars->q_full[nx % kQStages], (nx / kQStages) & 1, w))) break;
+          if (!(ok = all(wait_bar(&bars->q_full[nx % kQStages], (nx / kQStages) & 1, w)))) break;
           tc_fence_after();
           auto dp = issue_sdp(nx);
-          if (!(ok = wait_bar(&bars->dq_empty[x], (it >> 1) & 1, w))) break;
+          if (!(ok = all(wait_bar(&bars->dq_empty[x], (it >> 1) & 1, w)))) break;
           tc_fence_after();
           dp();
-          mma_commit(&bars->dp_full[x]);
+          mma_commit(&bars->dp_full[x], leader);
         }
       }
-      mma_commit(&bars->acc_final);
-      mma_commit(&bars->drain);
-      drain_bar(&bars->drain, 0, w);
+      mma_commit(&bars->acc_final, leader);
+      mma_commit(&bars->drain, leader);
+      all(drain_bar(&bars->drain, 0, w));
     }
   } else if (warp < 8) {
     // ------------------------------------------- P^T and dS^T (key rows)
@@ -374,8 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < kQT / 32; ++c) {
         uint32_t sv[32], dv[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_ld32(tDP + c * 32, dv);
+        tmem_ld32_nowait(tS + c * 32, sv);
+        tmem_ld32_nowait(tDP + c * 32, dv);
+        tmem_ld_wait(sv);
+        tmem_ld_tie(dv);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int y = 0; y < 8; ++y) {
@@ -414,6 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P^T chunk -> columns [16c, 16c+16) of this buffer's dP^T columns
         // (their dP^T values were loaded by this or the previous chunk).
         tmem_st16(tDP + c * 16, pk);
+        // dS^T chunk -> columns [16c, 16c+16) of this buffer's S^T columns
+        // (their S^T values were loaded by this or the previous chunk): the
+        // A operand of dK += dS^T Q straight from tensor memory.
+        tmem_st16(tS + c * 16, dk);
         // dS^T chunk: queries [32c, 32c+32) of key row kr, 128-byte swizzled.
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -620,6 +670,16 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   // Causal units differ in length: keep strict longest-first order over all
   // KV heads. Non-causal units are equal: group KV heads for L2 locality.
   a.group = MASK == 1 ? a.BHkv : l2_head_group(static_cast<long long>(8) * (s.Hq / s.Hkv) * s.N * D, a.BHkv);
+  // Causal: strict longest-first order over all KV heads keeps the tail
+  // short but spreads the resident CTAs over every head, whose dQ
+  // accumulators, Q and dO then fall out of L2 between visits. When those
+  // (8 bytes per element of a KV group's query heads) exceed a share of L2
+  // and a head has enough key tiles for bands of 16 to stay longest-first
+  // overall, order by bands of 16 key tiles, head-major within a band
+  // (measured on B200, B=2 H=16 N=8192 d=128: +4.8% on this kernel; at
+  // N=2048 the head-major order costs more in tail than it saves).
+  const long long group_bytes = static_cast<long long>(8) * (s.Hq / s.Hkv) * s.N * D;
+  a.band = (MASK == 1 && a.nk >= 64 && group_bytes * a.BHkv > (48ll << 20)) ? 16 : 0;
   a.window = s.window < 0 ? 0x3fffffff : s.window;
   a.prefix = s.prefix;
   a.scale = s.scale;

@@ -233,30 +233,36 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
   } else if (warp == kDecMma) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
+    // The whole warp runs this loop (descriptors stay warp-uniform); the
+    // elected lane issues the tcgen05 instructions.
+    const bool leader = elect_one();
+    auto all = [](bool b) { return __all_sync(0xffffffffu, b); };
+    {
       constexpr uint32_t idesc_qk = idesc_bf16(kT, kT, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(kT, D, false, true);
-      const uint32_t sQ = smem_u32(smem + C::kOffQ);
-      const uint32_t sK = smem_u32(smem + C::kOffK);
-      const uint32_t sV = smem_u32(smem + C::kOffV);
+      // Operand descriptors computed once and stepped by byte offsets.
+      const uint64_t dQ = sdesc_sw128(smem_u32(smem + C::kOffQ), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(smem + C::kOffV), C::kBoxBytes, 1024);
+      auto ofs_kmaj = [](int k) { return static_cast<uint32_t>((k / 4) * C::kBoxBytes + (k % 4) * 32); };
       // S_t = Q K_t^T into S buffer (t - t_lo) & 1.
       auto issue_s = [&](const TileCursor& ta) -> bool {
         const int g = static_cast<int>(ta.t - t_lo);
         const int s = g % ST;
         const int qb = ta.e % QB;
-        if (ta.first(t_lo) && !wait_bar(&bars->q_full[qb], (ta.e / QB) & 1, w)) return false;
-        if (!wait_bar(&bars->k_full[s], (g / ST) & 1, w)) return false;
+        if (ta.first(t_lo) && !all(wait_bar(&bars->q_full[qb], (ta.e / QB) & 1, w))) return false;
+        if (!all(wait_bar(&bars->k_full[s], (g / ST) & 1, w))) return false;
         tc_fence_after();
-        const uint32_t qa = sQ + qb * C::kTileBytes;
-        const uint32_t ka = sK + s * C::kTileBytes;
+        const uint64_t qa = sdesc_step(dQ, qb * C::kTileBytes);
+        const uint64_t ka = sdesc_step(dK, s * C::kTileBytes);
         const uint32_t d_s = tmem + kColS + (g & 1) * kT;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k / 4) * C::kBoxBytes + (k % 4) * 32;
-          mma_ss(d_s, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
-        }
-        mma_commit(&bars->s_full[g & 1]);
-        if (ta.last()) mma_commit(&bars->q_empty[qb]);  // the segment's last read of its Q buffer
+        for (int k = 0; k < D / 16; k += 4)
+          mma_ss_x4(d_s, sdesc_step(qa, ofs_kmaj(k)), sdesc_step(qa, ofs_kmaj(k + 1)), sdesc_step(qa, ofs_kmaj(k + 2)),
+                    sdesc_step(qa, ofs_kmaj(k + 3)), sdesc_step(ka, ofs_kmaj(k)), sdesc_step(ka, ofs_kmaj(k + 1)),
+                    sdesc_step(ka, ofs_kmaj(k + 2)), sdesc_step(ka, ofs_kmaj(k + 3)), idesc_qk, k > 0, leader);
+        mma_commit(&bars->s_full[g & 1], leader);
+        if (ta.last()) mma_commit(&bars->q_empty[qb], leader);  // the segment's last read of its Q buffer
         return true;
       };
       // O += P_t V_t.
@@ -264,20 +270,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int g = static_cast<int>(ta.t - t_lo);
         const int s = g % ST;
         const int ob = ta.e % OB;
-        if (!wait_bar(&bars->p_ready, g & 1, w) || !wait_bar(&bars->v_full[s], (g / ST) & 1, w)) return false;
+        if (!all(wait_bar(&bars->p_ready, g & 1, w)) || !all(wait_bar(&bars->v_full[s], (g / ST) & 1, w))) return false;
         const bool first = ta.first(t_lo);
-        if (first && ta.e >= OB && !wait_bar(&bars->o_empty[ob], ((ta.e / OB) - 1) & 1, w)) return false;
+        if (first && ta.e >= OB && !all(wait_bar(&bars->o_empty[ob], ((ta.e / OB) - 1) & 1, w))) return false;
         tc_fence_after();
-        const uint32_t va = sV + s * C::kTileBytes;
+        const uint64_t va = sdesc_step(dV, s * C::kTileBytes);
         const uint32_t d_o = tmem + kColO + ob * D;
         const uint32_t a_p = tmem + kColP + (g & 1) * 64;
 #pragma unroll
-        for (int k = 0; k < kT / 16; ++k)
-          mma_ts(d_o, a_p + k * 8, sdesc_sw128(va + k * 2048, C::kBoxBytes, 1024), idesc_pv,
-                 (!first || k > 0) ? 1u : 0u);
-        mma_commit(&bars->kv_empty[s]);
-        mma_commit(&bars->pv_done);
-        if (ta.last()) mma_commit(&bars->o_full[ob]);
+        for (int k = 0; k < kT / 16; k += 4)
+          mma_ts_x4(d_o, a_p + k * 8, a_p + (k + 1) * 8, a_p + (k + 2) * 8, a_p + (k + 3) * 8,
+                    sdesc_step(va, k * 2048), sdesc_step(va, (k + 1) * 2048), sdesc_step(va, (k + 2) * 2048),
+                    sdesc_step(va, (k + 3) * 2048), idesc_pv, (!first || k > 0) ? 1u : 0u, leader);
+        mma_commit(&bars->kv_empty[s], leader);
+        mma_commit(&bars->pv_done, leader);
+        if (ta.last()) mma_commit(&bars->o_full[ob], leader);
         return true;
       };
       TileCursor cur(P, t_lo, t_hi), nxt(P, t_lo, t_hi);
@@ -293,8 +300,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
       }
       // All MMAs issued by this thread must finish before tensor memory is freed.
-      mma_commit(&bars->drain);
-      drain_bar(&bars->drain, 0, w);
+      mma_commit(&bars->drain, leader);
+      all(drain_bar(&bars->drain, 0, w));
     }
   } else {
     // ------------------------------------------------------------- softmax

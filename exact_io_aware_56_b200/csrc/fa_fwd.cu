@@ -35,6 +35,12 @@
 // complete the O_t accumulator holds every earlier product and may be
 // rescaled in place until the first half of P_t^(j+1) is handed back.
 //
+// At d = 64 tensor memory also holds a separate P_t ([384 + 64t, +64)), and
+// the MMA thread issues S_t^(j+1) as soon as the softmax has loaded S_t^j
+// (barrier s_free), before O_t += P_t^j V_j. The softmax then waits for
+// that product's completion (barrier pv_done) before it writes P_t^(j+1) or
+// rescales O_t, instead of relying on the order above.
+//
 // The exponentials are base 2: scores are scaled by scale*log2(e), and
 // L = (m + log2 l) * ln 2. A warp whose rows' maxima did not grow on a tile
 // skips the tensor-memory round trip of the O rescale.
@@ -45,14 +51,19 @@
 #include "fa_internal.h"
 #include "sm100.cuh"
 
+#ifndef FA_FWD_PINGPONG
+#define FA_FWD_PINGPONG 0
+#endif
+
 namespace fa {
 namespace {
 
 constexpr int kBM = 128;   // query rows per Q tile
 constexpr int kBN = 128;   // keys per K/V tile
 constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;   // Q and K
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;  // V
 // Rescale threshold (log2 units): a warp rescales its O rows only when some
 // row's running max grew by more than this. With the O residual (the
 // training path, whose backward forms D from O to ~16 bits) it is 0: every
@@ -86,15 +97,19 @@ struct FwdCfg {
   static constexpr int kElem = F8 ? 1 : 2;              // bytes per element
   static constexpr int kBoxCols = 128 / kElem;          // elements per 128-byte swizzle row
   static constexpr int kKStep = 32 / kElem;             // MMA K per instruction (16 bf16, 32 e4m3)
-  static constexpr int kStages = (D * kElem == 256) ? 2 : 4;
+  // K and V rings: K_j is free once both S products of tile j are issued,
+  // V_j only after both P V products, so K gets the deeper ring where
+  // shared memory is short (d = 128 in bf16: 3 K stages, 2 V stages).
+  static constexpr int kKStages = (D * kElem == 256) ? 3 : 4;
+  static constexpr int kVStages = (D * kElem == 256) ? 2 : 4;
   static constexpr int kBoxBytes = kBN * 128;           // one 128-byte-wide TMA box of a 128-row tile
   static constexpr int kBoxes = D * kElem / 128;
   static constexpr int kTileBytes = kBoxBytes * kBoxes;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = 2 * kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kBarBytes = 256;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -125,8 +140,10 @@ struct FwdArgs {
 
 struct FwdBars {
   uint64_t q_full;
-  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t s_full[2], p_ready[2][2], o_final[2];  // p_ready: [Q tile][half of P]
+  uint64_t s_free[2], pv_done[2];  // separate-P schedule (d = 64) only
+  uint64_t tok[2];                  // exponential-phase token of each softmax warpgroup
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -146,7 +163,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<D, F8>;
   static_assert(!F8 || MASK != 2, "FP8 mode covers the unmasked and causal forward");
-  constexpr int ST = C::kStages;
+  // Separate-P schedule: with d = 64 tensor memory has room for P next to S
+  // (S_t at [128t, 128t+128), O_t at [256 + 64t, ...), P_t at [384 + 64t,
+  // 384 + 64t + 64)), so S_t of the next key tile is computed as soon as
+  // the softmax has loaded S_t, while it still turns the scores into P, and
+  // the softmax warps never wait for P V and S to pass through the tensor
+  // pipe between tiles.
+  constexpr bool SEP = (D == 64) && !F8;
+  constexpr int KS = C::kKStages;  // K ring stages
+  constexpr int VS = C::kVStages;  // V ring stages
+  static_assert(KS <= 4 && VS <= 4, "barrier arrays hold four stages");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -191,16 +217,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_ready[t][0], kBM);
       mbar_init(&bars->p_ready[t][1], kBM);
       mbar_init(&bars->o_final[t], 1);
+      mbar_init(&bars->s_free[t], kBM);
+      mbar_init(&bars->pv_done[t], 1);
+      mbar_init(&bars->tok[t], kBM);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -221,14 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sV = smem_u32(smem + C::kOffV);
 
   if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------- Q, K producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      int k_last[ST], v_last[ST];
+      int k_last[KS];
 #pragma unroll
-      for (int s = 0; s < ST; ++s) k_last[s] = v_last[s] = -1;
+      for (int s = 0; s < KS; ++s) k_last[s] = -1;
       mbar_arrive_expect_tx(&bars->q_full, 2 * C::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
@@ -238,17 +269,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                       x * C::kBoxCols, q0 + t * kBM, bh);
       const int n = n_t[1];
       for (int j = 0; j < n; ++j) {
-        const int s = j % ST;
-        const int u = j / ST;
-        if (j >= ST && !wait_bar(&bars->kv_empty[s], (u - 1) & 1, w)) break;
-        if (!(a.ctl.fault == 1 && j == 0)) {
-          mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+        const int s = j % KS;
+        const int u = j / KS;
+        if (j >= KS && !wait_bar(&bars->k_empty[s], (u - 1) & 1, w)) break;
+        if (a.ctl.fault == 1 && j == 0) continue;  // test hook: K_0 never arrives
+        mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
 #pragma unroll
-          for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes,
-                        x * C::kBoxCols, key_tile(j) * kBN, kvh);
-          k_last[s] = u;
-        }
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes,
+                      x * C::kBoxCols, key_tile(j) * kBN, kvh);
+        k_last[s] = u;
+      }
+      // Every copy issued must land before the CTA may exit.
+      drain_bar(&bars->q_full, 0, w);
+#pragma unroll
+      for (int s = 0; s < KS; ++s)
+        if (k_last[s] >= 0) drain_bar(&bars->k_full[s], k_last[s] & 1, w);
+    }
+  } else if (warp == kVProducerWarp) {
+    // ----------------------------------------------------------- V producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmV);
+      int v_last[VS];
+#pragma unroll
+      for (int s = 0; s < VS; ++s) v_last[s] = -1;
+      const int n = n_t[1];
+      for (int j = 0; j < n; ++j) {
+        const int s = j % VS;
+        const int u = j / VS;
+        if (j >= VS && !wait_bar(&bars->v_empty[s], (u - 1) & 1, w)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
 #pragma unroll
         for (int x = 0; x < C::kBoxes; ++x)
@@ -256,92 +305,149 @@ __global__ void __launch_bounds__(kThreads, 1)
                       x * C::kBoxCols, key_tile(j) * kBN, kvh);
         v_last[s] = u;
       }
-      // Every copy issued must land before the CTA may exit.
-      drain_bar(&bars->q_full, 0, w);
 #pragma unroll
-      for (int s = 0; s < ST; ++s) {
-        if (k_last[s] >= 0) drain_bar(&bars->k_full[s], k_last[s] & 1, w);
+      for (int s = 0; s < VS; ++s)
         if (v_last[s] >= 0) drain_bar(&bars->v_full[s], v_last[s] & 1, w);
-      }
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
+    // The whole warp runs this loop (descriptors stay warp-uniform); the
+    // elected lane issues the tcgen05 instructions.
+    const bool leader = elect_one();
+    auto all = [](bool b) { return __all_sync(0xffffffffu, b); };
+    {
       constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(kBM, kBN, false, false) : idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(kBM, D, false, true) : idesc_bf16(kBM, D, false, true);
-      constexpr int KS = C::kKStep;
+      constexpr int KSTEP = C::kKStep;  // MMA K per instruction (16 bf16, 32 e4m3)
       const uint32_t tS[2] = {tmem, tmem + 128u};
+      // A operand (P) of O += P V: over S, or in its own columns (SEP).
+      const uint32_t tP[2] = {SEP ? tmem + 384u : tmem, SEP ? tmem + 448u : tmem + 128u};
       const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      // Operand descriptors computed once and stepped by byte offsets
+      // (sdesc_step): K step k of a K-major tile is 32 bytes within a
+      // 128-byte swizzle row, boxes kBoxBytes apart; of the MN-major V tile,
+      // KSTEP rows of 128 bytes.
+      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sV, C::kBoxBytes, 1024);
+      auto ofs_kmaj = [](int k) { return static_cast<uint32_t>((k / 4) * C::kBoxBytes + (k % 4) * 32); };
       auto issue_s = [&](int t, int j) {
-        const uint32_t qa = sQ + t * C::kTileBytes;
-        const uint32_t ka = sK + (j % ST) * C::kTileBytes;
-        // Each K step is 32 bytes of a 128-byte swizzle row (16 bf16 or 32 e4m3).
+        const uint64_t qa = sdesc_step(dQ, t * C::kTileBytes);
+        const uint64_t ka = sdesc_step(dK, (j % KS) * C::kTileBytes);
+        if constexpr (F8) {
+          // Each K step is 32 bytes of a 128-byte swizzle row (32 e4m3).
 #pragma unroll
-        for (int k = 0; k < D / KS; ++k) {
-          const uint32_t off = (k / 4) * C::kBoxBytes + (k % 4) * 32;
-          if constexpr (F8)
-            mma_ss_f8(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
-          else
-            mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk, k > 0);
+          for (int k = 0; k < D / KSTEP; ++k)
+            mma_ss_f8(tS[t], sdesc_step(qa, ofs_kmaj(k)), sdesc_step(ka, ofs_kmaj(k)), idesc_qk, k > 0, leader);
+        } else {
+#pragma unroll
+          for (int k = 0; k < D / KSTEP; k += 4)
+            mma_ss_x4(tS[t], sdesc_step(qa, ofs_kmaj(k)), sdesc_step(qa, ofs_kmaj(k + 1)),
+                      sdesc_step(qa, ofs_kmaj(k + 2)), sdesc_step(qa, ofs_kmaj(k + 3)), sdesc_step(ka, ofs_kmaj(k)),
+                      sdesc_step(ka, ofs_kmaj(k + 1)), sdesc_step(ka, ofs_kmaj(k + 2)),
+                      sdesc_step(ka, ofs_kmaj(k + 3)), idesc_qk, k > 0, leader);
         }
-        mma_commit(&bars->s_full[t]);
+        mma_commit(&bars->s_full[t], leader);
       };
       // Half h of P V: keys [64h, 64h + 64).
       auto issue_pv = [&](int t, int j, int h) {
-        const uint32_t va = sV + (j % ST) * C::kTileBytes;
-        // P: KS keys per step = 8 tensor-memory columns (bf16 pairs or e4m3
-        // quads); V: KS key rows of 128 bytes (MN-major).
-        constexpr int KH = kBN / KS / 2;
+        const uint64_t va = sdesc_step(dV, (j % VS) * C::kTileBytes);
+        // P: KSTEP keys per step = 8 tensor-memory columns (bf16 pairs or e4m3
+        // quads); V: KSTEP key rows of 128 bytes (MN-major).
+        constexpr int KH = kBN / KSTEP / 2;
+        if constexpr (F8) {
 #pragma unroll
-        for (int k = h * KH; k < h * KH + KH; ++k) {
-          if constexpr (F8)
-            mma_ts_f8(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * KS * 128, C::kBoxBytes, 1024), idesc_pv,
-                      (j > 0 || k > 0) ? 1u : 0u);
-          else
-            mma_ts(tO[t], tS[t] + k * 8, sdesc_sw128(va + k * KS * 128, C::kBoxBytes, 1024), idesc_pv,
-                   (j > 0 || k > 0) ? 1u : 0u);
+          for (int k = h * KH; k < h * KH + KH; ++k)
+            mma_ts_f8(tO[t], tP[t] + k * 8, sdesc_step(va, k * KSTEP * 128), idesc_pv, (j > 0 || k > 0) ? 1u : 0u,
+                      leader);
+        } else {
+          static_assert(F8 || KH == 4, "one group of four MMAs per half");
+          const int k = h * KH;
+          mma_ts_x4(tO[t], tP[t] + k * 8, tP[t] + (k + 1) * 8, tP[t] + (k + 2) * 8, tP[t] + (k + 3) * 8,
+                    sdesc_step(va, k * KSTEP * 128), sdesc_step(va, (k + 1) * KSTEP * 128),
+                    sdesc_step(va, (k + 2) * KSTEP * 128), sdesc_step(va, (k + 3) * KSTEP * 128), idesc_pv,
+                    (j > 0 || k > 0) ? 1u : 0u, leader);
         }
       };
       const int n0 = n_t[0], n1 = n_t[1];
-      bool ok = wait_bar(&bars->q_full, 0, w) && wait_bar(&bars->k_full[0], 0, w);
+      bool ok = all(wait_bar(&bars->q_full, 0, w)) && all(wait_bar(&bars->k_full[0], 0, w));
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
+        mma_commit(&bars->k_empty[0], leader);  // K_0 read by both S products
       }
       for (int j = 0; ok && j < n1; ++j) {
-        const int s = j % ST;
-        const uint32_t par = (j / ST) & 1;
+        const int s = j % VS;                   // V_j stage
+        const uint32_t par = (j / VS) & 1;
         const int jn = j + 1;
+        if constexpr (SEP) {
+          // S_t of tile j + 1 as soon as the softmax has loaded S_t of tile
+          // j; then this tile's P V. pv_done tells the softmax when P_t and
+          // O_t may be written again.
+          if (j < n0) {
+            if (jn < n0) {
+              if (!(ok = all(wait_bar(&bars->s_free[0], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
+                break;
+              tc_fence_after();
+              issue_s(0, jn);
+            }
+            if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
+            tc_fence_after();
+            issue_pv(0, j, 0);
+            if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
+            tc_fence_after();
+            issue_pv(0, j, 1);
+            mma_commit(&bars->pv_done[0], leader);
+            if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
+          }
+          if (jn < n1) {
+            if (!(ok = all(wait_bar(&bars->s_free[1], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
+              break;
+            tc_fence_after();
+            issue_s(1, jn);
+            mma_commit(&bars->k_empty[jn % KS], leader);
+          }
+          if (!(ok = all(wait_bar(&bars->p_ready[1][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
+          tc_fence_after();
+          issue_pv(1, j, 0);
+          if (!(ok = all(wait_bar(&bars->p_ready[1][1], j & 1, w)))) break;
+          tc_fence_after();
+          issue_pv(1, j, 1);
+          mma_commit(&bars->pv_done[1], leader);
+          mma_commit(&bars->v_empty[s], leader);
+          if (j == n1 - 1) mma_commit(&bars->o_final[1], leader);
+          continue;
+        }
         if (j < n0) {
-          if (!(ok = wait_bar(&bars->p_ready[0][0], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
+          if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
           tc_fence_after();
           issue_pv(0, j, 0);
-          if (!(ok = wait_bar(&bars->p_ready[0][1], j & 1, w))) break;
+          if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
           tc_fence_after();
           issue_pv(0, j, 1);
-          if (j == n0 - 1) mma_commit(&bars->o_final[0]);
+          if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
           if (jn < n0) {
-            if (!(ok = wait_bar(&bars->k_full[jn % ST], (jn / ST) & 1, w))) break;
+            if (!(ok = all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w)))) break;
             issue_s(0, jn);
           }
         }
-        if (!(ok = wait_bar(&bars->p_ready[1][0], j & 1, w) && wait_bar(&bars->v_full[s], par, w))) break;
+        if (!(ok = all(wait_bar(&bars->p_ready[1][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
         tc_fence_after();
         issue_pv(1, j, 0);
-        if (!(ok = wait_bar(&bars->p_ready[1][1], j & 1, w))) break;
+        if (!(ok = all(wait_bar(&bars->p_ready[1][1], j & 1, w)))) break;
         tc_fence_after();
         issue_pv(1, j, 1);
-        mma_commit(&bars->kv_empty[s]);
-        if (j == n1 - 1) mma_commit(&bars->o_final[1]);
+        mma_commit(&bars->v_empty[s], leader);
+        if (j == n1 - 1) mma_commit(&bars->o_final[1], leader);
         if (jn < n1) {
-          if (!(ok = wait_bar(&bars->k_full[jn % ST], (jn / ST) & 1, w))) break;
+          if (!(ok = all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w)))) break;
           issue_s(1, jn);
+          mma_commit(&bars->k_empty[jn % KS], leader);
         }
       }
       // All MMAs issued by this thread must finish before tensor memory is freed.
-      mma_commit(&bars->drain);
-      drain_bar(&bars->drain, 0, w);
+      mma_commit(&bars->drain, leader);
+      all(drain_bar(&bars->drain, 0, w));
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------- softmax
@@ -351,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q0 + t * kBM + r;          // query position
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128u;
+    const uint32_t tPw = SEP ? tmem + lane_off + 384u + t * 64u : tS;  // where this tile's P goes
     const uint32_t tO = tmem + lane_off + 256u + t * D;
     const int n = n_t[t];
     // FP8 mode: the scores come out of the MMA in units of sq * sk (the Q
@@ -366,12 +473,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -CUDART_INF_F;  // running max of scale*log2(e)*s
     float l = 0.f;            // running sum, relative to m
     bool ok = true;
+#if FA_FWD_PINGPONG
+    // The two softmax warpgroups take turns on the exponential unit: tile t
+    // computes the exponentials of its key tile k only after holding token
+    // tok[t] for the k-th time and then hands the turn to the other tile;
+    // everything else (tensor-memory loads, row maxima, O rescales, waits)
+    // overlaps the other tile's exponentials. Both take n_t[1] turns (tile
+    // 0 ends with an empty one when it has a key tile fewer), tile 1 gives
+    // tile 0 its first turn and skips the hand-over after its last.
+    const int n_turns = n_t[1];
+    if (t == 1) mbar_arrive(&bars->tok[0]);
+#endif
     for (int j = 0; j < n; ++j) {
       ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[t], j & 1, w));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[kBN];
       tmem_ld128(tS, sr);
+      if constexpr (SEP) {
+        // S_t is in registers: the MMA thread may compute the next tile's S_t.
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[t]);
+      }
       const float sl2 = F8 ? sl2_q * a.f8.sk[static_cast<size_t>(kvh) * a.nk + key_tile(j)] : sl2_q;
       if (MASK != 2) {
         if (j == n - 1) {
@@ -425,6 +548,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // FP8 mode writes P as e4m3 of 2^kF8Offset p (headroom against
       // underflow, exact to undo): the offset rides on the exponent.
       const float neg_m = ((MASK == 2 && m == -CUDART_INF_F) ? 0.f : -m) + (F8 ? kF8Offset : 0.f);
+      if constexpr (SEP) {
+        // P_t and O_t of the previous key tile must have passed through P V
+        // before this tile's P overwrites P_t or O_t is rescaled.
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, wait_bar(&bars->pv_done[t], (j - 1) & 1, w));
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
+#if FA_FWD_PINGPONG
+      if (rescale) {
+        // O holds every earlier product (see the ordering argument above);
+        // scale this row by alpha before any P V of this tile is added
+        // (16 columns at a time: the 128 scores are still in registers).
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o16[16];
+          tmem_ld16(tO + c * 16, o16);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o16[i] = __float_as_uint(__uint_as_float(o16[i]) * alpha);
+          tmem_st16(tO + c * 16, o16);
+        }
+      }
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->tok[t], j & 1, w));
+      if (!ok) break;
+#endif
       float ps[8];  // 8 independent partial row sums
 #pragma unroll
       for (int u = 0; u < 8; ++u) ps[u] = 0.f;
@@ -453,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             pk[i] = pack_e4m3x4(p4[0], p4[1], p4[2], p4[3]);
           }
-          tmem_st16(tS + c * 16, pk);
+          tmem_st16(tPw + c * 16, pk);
         } else {
 #pragma unroll
           for (int c = 2 * h; c < 2 * h + 2; ++c) {
@@ -470,9 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               fadd2(ps[(2 * i) & 7], ps[(2 * i + 1) & 7], ps[(2 * i) & 7], ps[(2 * i + 1) & 7], p0, p1);
               pk[i] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(tS + c * 16, pk);
+            tmem_st16(tPw + c * 16, pk);
           }
         }
+#if !FA_FWD_PINGPONG
         if (h == 0 && rescale) {
           // O holds every earlier product (see the ordering argument above);
           // scale this row by alpha before P V is added to it.
@@ -485,12 +635,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + c * 32, o32);
           }
         }
+#endif
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_ready[t][h]);
       }
+#if FA_FWD_PINGPONG
+      if (!(t == 1 && j == n_turns - 1)) mbar_arrive(&bars->tok[1 - t]);
+#endif
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
     }
+#if FA_FWD_PINGPONG
+    // Tile 0 with a key tile fewer: its last turn is empty.
+    if (ok && t == 0 && n < n_turns) {
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->tok[0], n & 1, w));
+      if (ok) mbar_arrive(&bars->tok[1]);
+    }
+#endif
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->o_final[t], 0, w));
     if (ok) {
       tc_fence_after();

@@ -41,6 +41,14 @@ def _record(name, diff, ref, excess, extra_max=0.0):
         f.write(json.dumps(line) + "\n")
 
 
+def record_bound(name, err, ref, bound):
+    """Appends one report line (see FA_PARITY_REPORT) for a comparison that
+    a test checks against its own elementwise ``bound``."""
+    err, ref, bound = (np.asarray(x, dtype=np.float64) for x in (err, ref, bound))
+    if err.size:
+        _record(name, err, ref, (err - bound).max(), bound.max())
+
+
 def assert_close_abs(name, got, ref, tol=TOL_ABS, extra=0.0):
     """|got - ref| <= tol + 2^-8 |ref| (+ ``extra``, an elementwise bound on
     errors the inputs carry in, where a test derives one) everywhere."""

@@ -26,7 +26,7 @@ import torch
 import oracle
 from exact_io_aware_56_b200 import FP8_WORKLOADS, fa, make_inputs, sample_rows, to_f64
 
-from .parity import assert_close_lse
+from .parity import assert_close_lse, record_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -179,6 +179,7 @@ def _check_fp8_workload(name, rows_per_head):
             bound = fp8_bound(qh[b:b + 1, h:h + 1], kh[b:b + 1, g:g + 1], vh[b:b + 1, g:g + 1], w.causal, w.scale,
                               O[None, None], rows)[0, 0]
             err = np.abs(o[b, h, rows] - O)
+            record_bound(f"O[{b},{h}]", err, O, bound)
             assert np.isfinite(o[b, h, rows]).all(), (b, h)
             assert (err <= bound).all(), (b, h, float((err - bound).max()), float(err.max()))
             assert_close_lse(lse[b, h, rows], L)
