@@ -51,10 +51,6 @@
 #include "fa_internal.h"
 #include "sm100.cuh"
 
-#ifndef FA_FWD_PINGPONG
-#define FA_FWD_PINGPONG 0
-#endif
-
 namespace fa {
 namespace {
 
@@ -109,7 +105,7 @@ struct FwdCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kBarBytes = 512;
+  static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -143,7 +139,6 @@ struct FwdBars {
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t s_full[2], p_ready[2][2], o_final[2];  // p_ready: [Q tile][half of P]
   uint64_t s_free[2], pv_done[2];  // separate-P schedule (d = 64) only
-  uint64_t tok[2];                  // exponential-phase token of each softmax warpgroup
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -232,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->o_final[t], 1);
       mbar_init(&bars->s_free[t], kBM);
       mbar_init(&bars->pv_done[t], 1);
-      mbar_init(&bars->tok[t], kBM);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -473,17 +467,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -CUDART_INF_F;  // running max of scale*log2(e)*s
     float l = 0.f;            // running sum, relative to m
     bool ok = true;
-#if FA_FWD_PINGPONG
-    // The two softmax warpgroups take turns on the exponential unit: tile t
-    // computes the exponentials of its key tile k only after holding token
-    // tok[t] for the k-th time and then hands the turn to the other tile;
-    // everything else (tensor-memory loads, row maxima, O rescales, waits)
-    // overlaps the other tile's exponentials. Both take n_t[1] turns (tile
-    // 0 ends with an empty one when it has a key tile fewer), tile 1 gives
-    // tile 0 its first turn and skips the hand-over after its last.
-    const int n_turns = n_t[1];
-    if (t == 1) mbar_arrive(&bars->tok[0]);
-#endif
     for (int j = 0; j < n; ++j) {
       ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[t], j & 1, w));
       if (!ok) break;
@@ -557,23 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
       }
-#if FA_FWD_PINGPONG
-      if (rescale) {
-        // O holds every earlier product (see the ordering argument above);
-        // scale this row by alpha before any P V of this tile is added
-        // (16 columns at a time: the 128 scores are still in registers).
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o16[16];
-          tmem_ld16(tO + c * 16, o16);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o16[i] = __float_as_uint(__uint_as_float(o16[i]) * alpha);
-          tmem_st16(tO + c * 16, o16);
-        }
-      }
-      ok = __all_sync(0xffffffffu, wait_bar(&bars->tok[t], j & 1, w));
-      if (!ok) break;
-#endif
       float ps[8];  // 8 independent partial row sums
 #pragma unroll
       for (int u = 0; u < 8; ++u) ps[u] = 0.f;
@@ -622,7 +588,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tPw + c * 16, pk);
           }
         }
-#if !FA_FWD_PINGPONG
         if (h == 0 && rescale) {
           // O holds every earlier product (see the ordering argument above);
           // scale this row by alpha before P V is added to it.
@@ -635,23 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + c * 32, o32);
           }
         }
-#endif
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_ready[t][h]);
       }
-#if FA_FWD_PINGPONG
-      if (!(t == 1 && j == n_turns - 1)) mbar_arrive(&bars->tok[1 - t]);
-#endif
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
     }
-#if FA_FWD_PINGPONG
-    // Tile 0 with a key tile fewer: its last turn is empty.
-    if (ok && t == 0 && n < n_turns) {
-      ok = __all_sync(0xffffffffu, wait_bar(&bars->tok[0], n & 1, w));
-      if (ok) mbar_arrive(&bars->tok[1]);
-    }
-#endif
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->o_final[t], 0, w));
     if (ok) {
       tc_fence_after();
