@@ -23,6 +23,10 @@ __global__ void test_exp2_kernel(const float* x, float* yp, float* ye, int n) {
   }
 }
 
+__global__ void test_exp2_accurate_kernel(const float* x, float* y, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) y[i] = exp2_accurate(x[i]);
+}
+
 constexpr int kMaxDevices = 64;
 
 // Device error word written by the kernels' watchdog.
@@ -383,6 +387,15 @@ int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* strea
   if (n == 0) return FA_OK;
   const int blocks = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
   test_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_ex2, n);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : record_cuda(e);
+}
+
+int fa_test_exp2_accurate(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 0) return FA_ERR_INVALID_ARGUMENT;
+  if (n == 0) return FA_OK;
+  const int blocks = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
+  test_exp2_accurate_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }

@@ -84,7 +84,8 @@ constexpr float kF8Offset = 8.0f - kF8Rescale;
 // (exp2_poly) and the rest on the exponential unit. Measured on B200 at
 // N = 8192, d = 128: 0 of 32 is fastest (4, 8, 12 cost 3%, 8%, 14%): the
 // softmax warps are bound by instruction issue, not by the exponential unit,
-// so the extra FMA-pipe instructions only add issue slots.
+// so the extra FMA-pipe instructions only add issue slots. FP8 mode likewise
+// (4 of 16: +0.5%, within noise; 8 of 16: -12%).
 constexpr int kPolyPer32 = 0;
 
 // F8: e4m3 Q, K, V with block scales (the FP8 mode); otherwise bf16.
@@ -521,7 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_cand;  // -inf for a row with no visible key yet (mask kind 2)
       } else if (__any_sync(0xffffffffu, m_cand > m + a.rescale_tau)) {
         const float m_new = fmaxf(m, m_cand);
-        alpha = (MASK == 2 && m_new == -CUDART_INF_F) ? 1.f : ex2(m - m_new);
+        // On the FMA pipe: an ex2 here would queue behind the other tile's
+        // exponentials on the exponential unit.
+        alpha = (MASK == 2 && m_new == -CUDART_INF_F) ? 1.f : exp2_accurate(m - m_new);
         m = m_new;
         l *= alpha;
         rescale = true;
@@ -590,7 +593,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (h == 0 && rescale) {
           // O holds every earlier product (see the ordering argument above);
-          // scale this row by alpha before P V is added to it.
+          // scale this row by alpha before P V is added to it (32 columns
+          // per tensor-memory round trip: more would spill at d = 128, where
+          // 64 scores are still live here).
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o32[32];

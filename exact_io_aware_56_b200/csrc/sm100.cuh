@@ -409,6 +409,26 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x < -125.f ? 0.f : y;
 }
 
+// 2^x for x <= 0 on the FMA pipe to float32 accuracy (the degree-6
+// polynomial of exp2_poly.h, same range reduction as exp2_poly). Used for
+// the O rescale factor, one per row and key tile, which would otherwise
+// queue on the exponential unit behind the other softmax warpgroup's
+// weights. Arguments below -125 (and -inf) give exactly 0.
+__device__ __forceinline__ float exp2_accurate(float x) {
+  x = fmaxf(x, -127.f);
+  const float r = __fadd_rn(x, 12582912.f);
+  const float n = __fadd_rn(r, -12582912.f);
+  const float f = __fadd_rn(x, -n);
+  float p = fmaf(kExp2A6, f, kExp2A5);
+  p = fmaf(p, f, kExp2A4);
+  p = fmaf(p, f, kExp2A3);
+  p = fmaf(p, f, kExp2A2);
+  p = fmaf(p, f, kExp2A1);
+  p = fmaf(p, f, kExp2A0);
+  const float y = __uint_as_float(__float_as_uint(p) + (__float_as_uint(r) << 23));
+  return x < -125.f ? 0.f : y;
+}
+
 // Two fp32 fused multiply-adds in one instruction (sm_100 packed f32x2).
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
                                       float c1) {

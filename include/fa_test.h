@@ -33,6 +33,14 @@ void fa_test_set_fault(int code);
 int fa_test_exp2(const float* x, float* y_poly, float* y_ex2, int n, void* stream);
 
 /*
+ * Evaluates, for n device floats x (each <= 0), the forward kernel's
+ * float32-accurate FMA-pipe exponential (the one it uses for the O rescale
+ * factor) into y (n device floats), asynchronously on `stream`. Returns
+ * FA_OK, FA_ERR_INVALID_ARGUMENT (null pointer, n < 0) or FA_ERR_CUDA.
+ */
+int fa_test_exp2_accurate(const float* x, float* y, int n, void* stream);
+
+/*
  * Host only (no device call): the stream-K work partition fa_decode would
  * use for this shape with num_ctas CTAs, as eight integers in out[0..7]:
  * W (key tiles over all units), T (128-key tiles per unit), G (CTAs = runs),
