@@ -184,14 +184,16 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, void* 
   if (rc != FA_OK) return rc;
   DevState* st = nullptr;
   if ((rc = device_state(&st)) != FA_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to, tr;
   if (!encode_tile_map(&tq, q, d, N, B * Hq, 128) || !encode_tile_map(&tk, k, d, N, B * Hkv, 128) ||
-      !encode_tile_map(&tv, v, d, N, B * Hkv, 128))
+      !encode_tile_map(&tv, v, d, N, B * Hkv, 128) || !encode_tile_map(&to, o, d, N, B * Hq, 128) ||
+      !encode_tile_map(&tr, o_resid ? o_resid : o, d, N, B * Hq, 128))
     return FA_ERR_UNSUPPORTED;
   AttnShape s{B, Hq, Hkv, N, d, causal, scale};
   s.window = window;
   s.prefix = prefix;
-  cudaError_t e = launch_fwd(s, tq, tk, tv, o, o_resid, lse, make_ctl(st), static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_fwd(s, tq, tk, tv, to, tr, o, o_resid, lse, make_ctl(st), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
 
@@ -295,13 +297,15 @@ int fa_fwd_fp8(const void* q8, const float* sq, const void* k8, const float* sk,
   DevState* st = nullptr;
   if ((rc = device_state(&st)) != FA_OK) return rc;
   // e4m3 tensors: 128 one-byte columns per row, boxes of 128 columns x 128 rows.
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q8, d, N, B * Hq, 128, 128) ||
       !encode_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k8, d, N, B * Hkv, 128, 128) ||
-      !encode_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v8, d, N, B * Hkv, 128, 128))
+      !encode_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v8, d, N, B * Hkv, 128, 128) ||
+      !encode_tile_map(&to, o, d, N, B * Hq, 128))
     return FA_ERR_UNSUPPORTED;
   AttnShape s{B, Hq, Hkv, N, d, causal, scale};
-  cudaError_t e = launch_fwd_fp8(s, tq, tk, tv, o, lse, sq, sk, sv, make_ctl(st), static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_fwd_fp8(s, tq, tk, tv, to, o, lse, sq, sk, sv, make_ctl(st), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }
 

@@ -44,6 +44,10 @@
 // The exponentials are base 2: scores are scaled by scale*log2(e), and
 // L = (m + log2 l) * ln 2. A warp whose rows' maxima did not grow on a tile
 // skips the tensor-memory round trip of the O rescale.
+//
+// Epilogue (bf16 mode): each softmax warpgroup stages its normalised O tile
+// (and the residual) in shared memory in the 128-byte-swizzled box layout
+// and writes it with TMA tensor stores (o and o_resid tensor maps).
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -106,8 +110,13 @@ struct FwdCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kBarBytes = 512;
+  // Output staging (the epilogue, bf16 mode): two 16-KB boxes per Q tile.
+  // Where a Q tile is smaller than that (d = 64) they get their own region;
+  // otherwise the finished Q_t buffer holds them.
+  static constexpr bool kOwnStage = !F8 && kTileBytes < 2 * 16384;
+  static constexpr int kOffStage = (kOffBar + kBarBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmemBytes = (kOwnStage ? kOffStage + 4 * 16384 : kOffBar + kBarBytes) + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(kSmemBytes > 114 * 1024, "one CTA per SM (owns all tensor memory)");
@@ -122,8 +131,8 @@ struct Fp8Scales {
 };
 
 struct FwdArgs {
-  __nv_bfloat16* o;
-  __nv_bfloat16* o_resid;  // optional: bf16(O - bf16(O)), the rounding residual of o
+  void* o;              // stored through tmO, except in FP8 mode
+  const void* o_resid;  // optional: bf16(O - bf16(O)), the rounding residual of o (stored through tmR)
   float* lse;
   int N, Hq, Hkv, BH, n_pairs, nk;
   int group;  // heads per scheduling group (see the work-unit comment)
@@ -140,6 +149,7 @@ struct FwdBars {
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t s_full[2], p_ready[2][2], o_final[2];  // p_ready: [Q tile][half of P]
   uint64_t s_free[2], pv_done[2];  // separate-P schedule (d = 64) only
+  uint64_t epi_full[2], epi_free[2];  // output staging (see the epilogue)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -156,7 +166,8 @@ __device__ __forceinline__ bool visible2(int i, int j, int window, int prefix) {
 template <int D, int MASK, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const __grid_constant__ CUtensorMap tmR, const FwdArgs a) {
   using C = FwdCfg<D, F8>;
   static_assert(!F8 || MASK != 2, "FP8 mode covers the unmasked and causal forward");
   // Separate-P schedule: with d = 64 tensor memory has room for P next to S
@@ -228,6 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->o_final[t], 1);
       mbar_init(&bars->s_free[t], kBM);
       mbar_init(&bars->pv_done[t], 1);
+      mbar_init(&bars->epi_full[t], kBM);
+      mbar_init(&bars->epi_free[t], 1);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -617,31 +630,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       // FP8 mode: l sums 2^kF8Offset p, O sums the same weights times V's
       // codes; V's head scale turns codes into values.
       const float inv_l = F8 ? a.f8.sv[kvh] / l : 1.f / l;
-      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.N + row) * D;
-      __nv_bfloat16* rrow = a.o_resid ? a.o_resid + (static_cast<size_t>(bh) * a.N + row) * D : nullptr;
+      if constexpr (!F8) {
+        // O (then its residual) leaves through two staging boxes (the Q_t
+        // buffer, which no MMA reads any more, where it is large enough):
+        // each job is one 64-column box of 128 rows, written by the rows'
+        // threads in the tensor map's 128-byte swizzle and stored by one TMA
+        // copy, so that global memory sees whole lines (one thread per row
+        // storing its own row writes half sectors; measured on B200 the
+        // staged form takes ~6000 cycles off each CTA's epilogue at d = 128
+        // with the residual). Rows past N are clipped by the copy; a tile
+        // that starts past N has no job.
+        constexpr int kBoxesO = D / 64;  // bf16 output boxes
+        constexpr int kSlots = 2;        // 16-KB boxes staged at a time
+        const int jobs = qt0 < a.N ? kBoxesO * (a.o_resid ? 2 : 1) : 0;
+        uint8_t* stage = C::kOwnStage ? smem + C::kOffStage + t * 2 * 16384 : smem + C::kOffQ + t * C::kTileBytes;
+        const bool issuer = r == 0;
+        for (int i = 0; i < jobs; ++i) {
+          const int x = i % kBoxesO;
+          const bool resid = i >= kBoxesO;
+          uint8_t* slot = stage + (i % kSlots) * 16384;
+          // The slot's previous box must have been read by its copy.
+          if (i >= kSlots && !(ok = __all_sync(0xffffffffu, wait_bar(&bars->epi_free[t], (i - kSlots) & 1, w)))) break;
+          uint32_t oo[64];
+          uint32_t(&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oo[0]);
+          uint32_t(&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oo[32]);
+          tmem_ld32_nowait(tO + x * 64, o0);
+          tmem_ld32_nowait(tO + x * 64 + 32, o1);
+          tmem_ld_wait(o0);
+          tmem_ld_tie(o1);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t oo[32];
-        tmem_ld32(tO + c * 32, oo);
-        uint4 v[4], res[4];
-        uint32_t* pv = reinterpret_cast<uint32_t*>(v);
-        uint32_t* pr = reinterpret_cast<uint32_t*>(res);
+          for (int cc = 0; cc < 8; ++cc) {
+            uint4 v;
+            uint32_t* pv = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float x0 = __uint_as_float(oo[2 * i]) * inv_l;
-          const float x1 = __uint_as_float(oo[2 * i + 1]) * inv_l;
-          pv[i] = pack_bf16x2(x0, x1);
-          const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pv[i]);
-          pr[i] = pack_bf16x2(x0 - __low2float(hi), x1 - __high2float(hi));
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = __uint_as_float(oo[8 * cc + 2 * e]) * inv_l;
+              const float x1 = __uint_as_float(oo[8 * cc + 2 * e + 1]) * inv_l;
+              pv[e] = pack_bf16x2(x0, x1);
+              if (resid) {
+                const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&pv[e]);
+                pv[e] = pack_bf16x2(x0 - __low2float(hi), x1 - __high2float(hi));
+              }
+            }
+            *reinterpret_cast<uint4*>(slot + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->epi_full[t]);
+          if (issuer) {
+            if (!(ok = wait_bar(&bars->epi_full[t], i & 1, w))) break;
+            tma_store_3d(resid ? &tmR : &tmO, slot, x * 64, qt0, bh);
+            bulk_commit();
+            if (i + 1 < jobs && i + 1 >= kSlots) {
+              bulk_wait_read<kSlots - 1>();
+              mbar_arrive(&bars->epi_free[t]);
+            }
+          }
         }
-        if (row < a.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        // The copies must have read the staged boxes before the CTA exits.
+        if (issuer) bulk_wait_read<0>();
+      } else {
+        // FP8 mode (no residual): one thread per row stores its own row
+        // (measured on B200: staging costs 1 to 2% here).
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (static_cast<size_t>(bh) * a.N + row) * D;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = v[i];
-          if (rrow) {
-            uint4* rd = reinterpret_cast<uint4*>(rrow + c * 32);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t oo[32];
+          tmem_ld32(tO + c * 32, oo);
+          uint4 v[4];
+          uint32_t* pv = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rd[i] = res[i];
+          for (int i = 0; i < 16; ++i)
+            pv[i] = pack_bf16x2(__uint_as_float(oo[2 * i]) * inv_l, __uint_as_float(oo[2 * i + 1]) * inv_l);
+          if (row < a.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = v[i];
           }
         }
       }
@@ -661,15 +724,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, int MASK, bool F8 = false>
 cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream,
+                         const CUtensorMap& to, const CUtensorMap& tr, void* o, void* o_resid, float* lse,
+                         const LaunchCtl& ctl, cudaStream_t stream,
                          Fp8Scales f8 = Fp8Scales{nullptr, nullptr, nullptr}) {
   using C = FwdCfg<D, F8>;
   auto kern = fwd_kernel<D, MASK, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   FwdArgs a;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  a.o_resid = static_cast<__nv_bfloat16*>(o_resid);
+  a.o = o;
+  a.o_resid = o_resid;
   a.lse = lse;
   a.N = s.N;
   a.Hq = s.Hq;
@@ -689,15 +753,16 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.n_pairs) * a.BH;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, tr, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream) {
-#define FA_FWD_ARGS s, tq, tk, tv, o, o_resid, lse, ctl, stream
+                       const CUtensorMap& to, const CUtensorMap& tr, void* o, void* o_resid, float* lse,
+                       const LaunchCtl& ctl, cudaStream_t stream) {
+#define FA_FWD_ARGS s, tq, tk, tv, to, tr, o, o_resid, lse, ctl, stream
   switch (s.mask_kind() + (s.d == 64 ? 0 : 3)) {
     case 0: return launch_fwd_t<64, 0>(FA_FWD_ARGS);
     case 1: return launch_fwd_t<64, 1>(FA_FWD_ARGS);
@@ -710,12 +775,12 @@ cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensor
 }
 
 cudaError_t launch_fwd_fp8(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           void* o, float* lse, const float* sq, const float* sk, const float* sv,
-                           const LaunchCtl& ctl, cudaStream_t stream) {
+                           const CUtensorMap& to, void* o, float* lse, const float* sq, const float* sk,
+                           const float* sv, const LaunchCtl& ctl, cudaStream_t stream) {
   if (s.d != 128 || s.mask_kind() == 2) return cudaErrorInvalidValue;
   const Fp8Scales f8{sq, sk, sv};
-  if (s.causal) return launch_fwd_t<128, 1, true>(s, tq, tk, tv, o, nullptr, lse, ctl, stream, f8);
-  return launch_fwd_t<128, 0, true>(s, tq, tk, tv, o, nullptr, lse, ctl, stream, f8);
+  if (s.causal) return launch_fwd_t<128, 1, true>(s, tq, tk, tv, to, to, o, nullptr, lse, ctl, stream, f8);
+  return launch_fwd_t<128, 0, true>(s, tq, tk, tv, to, to, o, nullptr, lse, ctl, stream, f8);
 }
 
 }  // namespace fa

@@ -56,15 +56,18 @@ int check_current_device();
 // FA_ERR_CUDA.
 int record_cuda_error(cudaError_t e);
 
-// o_resid may be null (no residual written).
+// o_resid may be null (no residual written). to and tr are bf16 tensor maps
+// of o and o_resid laid out like q (tr unused without a residual).
 cudaError_t launch_fwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       void* o, void* o_resid, float* lse, const LaunchCtl& ctl, cudaStream_t stream);
+                       const CUtensorMap& to, const CUtensorMap& tr, void* o, void* o_resid, float* lse,
+                       const LaunchCtl& ctl, cudaStream_t stream);
 
 // FP8 mode (d = 128, masks 0 and 1): q, k, v are e4m3 codes behind 1-byte
-// tensor maps with 128-column boxes; sq, sk, sv the block scales.
+// tensor maps with 128-column boxes; sq, sk, sv the block scales; to the
+// bf16 tensor map of o.
 cudaError_t launch_fwd_fp8(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           void* o, float* lse, const float* sq, const float* sk, const float* sv,
-                           const LaunchCtl& ctl, cudaStream_t stream);
+                           const CUtensorMap& to, void* o, float* lse, const float* sq, const float* sk,
+                           const float* sv, const LaunchCtl& ctl, cudaStream_t stream);
 
 // e4m3 block quantization of a bf16 tensor [BH][N][d]: scales per 128-row
 // block ([BH][ceil(N/128)]) or per head ([BH]); see fa.h.
