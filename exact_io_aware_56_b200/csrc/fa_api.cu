@@ -232,11 +232,12 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   DevState* st = nullptr;
   if ((rc = device_state(&st)) != FA_OK) return rc;
   // The backward streams 64-row query tiles past 128-row key tiles.
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if (!encode_tile_map(&tq, q, d, N, B * Hq, 64) || !encode_tile_map(&tk, k, d, N, B * Hkv, 128) ||
-      !encode_tile_map(&tv, v, d, N, B * Hkv, 128) || !encode_tile_map(&tdo, dout, d, N, B * Hq, 64))
+      !encode_tile_map(&tv, v, d, N, B * Hkv, 128) || !encode_tile_map(&tdo, dout, d, N, B * Hq, 64) ||
+      !encode_tile_map(&tdk, dk, d, N, B * Hkv, 128) || !encode_tile_map(&tdv, dv, d, N, B * Hkv, 128))
     return FA_ERR_UNSUPPORTED;
-  cudaError_t e = launch_bwd(s, tq, tk, tv, tdo, o, o_resid, dout, lse, dq, dk, dv, workspace, make_ctl(st),
+  cudaError_t e = launch_bwd(s, tq, tk, tv, tdo, tdk, tdv, o, o_resid, dout, lse, dq, dk, dv, workspace, make_ctl(st),
                              static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : record_cuda(e);
 }

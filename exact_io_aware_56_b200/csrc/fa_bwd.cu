@@ -100,8 +100,6 @@ struct BwdArgs {
   const float* lse;
   const float* dsum;    // D_i, fp32 [B*Hq*N]
   float* dq_acc;        // fp32 [B*Hq*N*d]
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
   int N, Hq, Hkv, BHkv, nk, nq;
   int group;  // KV heads per scheduling group (see the work-unit comment)
   int band;   // causal: key tiles per scheduling band (0: strict longest-first)
@@ -116,6 +114,7 @@ struct BwdBars {
   uint64_t q_full[kQStages], q_empty[kQStages];
   uint64_t s_full[2], dp_full[2], p_ready[2], ds_free[2], dq_full[2], dq_empty[2];
   uint64_t acc_final, drain;
+  uint64_t epi_dv, epi_dk;  // output staging: all rows of dV / dK written to shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -135,6 +134,7 @@ template <int D, int MASK>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                     const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->acc_final, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->epi_dv, 256);
+    mbar_init(&bars->epi_dk, 128);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -477,26 +479,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars->p_ready[x]);
     }
-    // Epilogue: dV_j rows (this thread's key row), half of the columns per warpgroup.
+    // Epilogue: dV_j rows (this thread's key row), half of the columns per
+    // warpgroup, staged over V_j (no MMA reads it any more) in its 128-byte
+    // swizzled box layout and written by TMA stores once all 256 threads
+    // have staged theirs (whole lines instead of one thread per row writing
+    // half sectors). Key rows past N are clipped by the copy.
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
       tc_fence_after();
-      const int key = j * kKT + kr;
-      __nv_bfloat16* dst = a.dv + (static_cast<size_t>(bkv) * a.N + key) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
-        const int c = x * (D / 64) + cc;
+        const int c = x * (D / 64) + cc;  // 32-column chunk
         uint32_t vv[32];
         tmem_ld32(tmem + lane_off + C::kColDV + c * 32, vv);
-        uint4 o4[4];
-        uint32_t* po = reinterpret_cast<uint32_t*>(o4);
+        uint8_t* row = smem + C::kOffV + (c / 2) * C::kKBox + kr * 128;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) po[e] = pack_bf16x2(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1]));
-        if (key < a.N) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(dst + c * 32)[e] = o4[e];
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t chunk = static_cast<uint32_t>((c % 2) * 4 + u);
+          *reinterpret_cast<uint4*>(row + ((chunk ^ (kr & 7)) << 4)) =
+              make_uint4(pack_bf16x2(__uint_as_float(vv[8 * u]), __uint_as_float(vv[8 * u + 1])),
+                         pack_bf16x2(__uint_as_float(vv[8 * u + 2]), __uint_as_float(vv[8 * u + 3])),
+                         pack_bf16x2(__uint_as_float(vv[8 * u + 4]), __uint_as_float(vv[8 * u + 5])),
+                         pack_bf16x2(__uint_as_float(vv[8 * u + 6]), __uint_as_float(vv[8 * u + 7])));
         }
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->epi_dv);
+      if (threadIdx.x == 0 && wait_bar(&bars->epi_dv, 0, w)) {
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmDV, smem + C::kOffV + b * C::kKBox, b * 64, j * kKT, bkv);
+        bulk_commit();
+      }
+      if (threadIdx.x == 0) bulk_wait_read<0>();
     }
   } else if (warp >= kDqWarp0) {
     // ------------------------------------------- dQ_i^T readout (columns of dQ)
@@ -542,26 +556,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // Epilogue: dK_j = scale * accumulated dS^T Q (row m = key row).
+    // Epilogue: dK_j = scale * accumulated dS^T Q (row m = key row), staged
+    // over K_j and written by TMA stores as dV is.
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(&bars->acc_final, 0, w));
     if (ok) {
       tc_fence_after();
-      const int key = j * kKT + m;
-      __nv_bfloat16* dst = a.dk + (static_cast<size_t>(bkv) * a.N + key) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t vv[32];
         tmem_ld32(tmem + lane_off + C::kColDK + c * 32, vv);
-        uint4 o4[4];
-        uint32_t* po = reinterpret_cast<uint32_t*>(o4);
+        uint8_t* row = smem + C::kOffK + (c / 2) * C::kKBox + m * 128;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          po[e] = pack_bf16x2(__uint_as_float(vv[2 * e]) * a.scale, __uint_as_float(vv[2 * e + 1]) * a.scale);
-        if (key < a.N) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(dst + c * 32)[e] = o4[e];
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t chunk = static_cast<uint32_t>((c % 2) * 4 + u);
+          *reinterpret_cast<uint4*>(row + ((chunk ^ (m & 7)) << 4)) = make_uint4(
+              pack_bf16x2(__uint_as_float(vv[8 * u]) * a.scale, __uint_as_float(vv[8 * u + 1]) * a.scale),
+              pack_bf16x2(__uint_as_float(vv[8 * u + 2]) * a.scale, __uint_as_float(vv[8 * u + 3]) * a.scale),
+              pack_bf16x2(__uint_as_float(vv[8 * u + 4]) * a.scale, __uint_as_float(vv[8 * u + 5]) * a.scale),
+              pack_bf16x2(__uint_as_float(vv[8 * u + 6]) * a.scale, __uint_as_float(vv[8 * u + 7]) * a.scale));
         }
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->epi_dk);
+      const bool issuer = warp == kDqWarp0 && lane == 0;
+      if (issuer && wait_bar(&bars->epi_dk, 0, w)) {
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmDK, smem + C::kOffK + b * C::kKBox, b * 64, j * kKT, bkv);
+        bulk_commit();
+      }
+      if (issuer) bulk_wait_read<0>();
     }
   }
 
@@ -636,9 +659,9 @@ int grid_for(long long work, int per_block, int cap) {
 
 template <int D, int MASK>
 cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
-                         const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
-                         cudaStream_t stream) {
+                         const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const void* o,
+                         const void* o_resid, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         void* workspace, const LaunchCtl& ctl, cudaStream_t stream) {
   using C = BwdCfg<D>;
   const long long rows = static_cast<long long>(s.B) * s.Hq * s.N;
   float* dsum = static_cast<float*>(workspace);
@@ -659,8 +682,8 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.lse = lse;
   a.dsum = dsum;
   a.dq_acc = dq_acc;
-  a.dk = static_cast<__nv_bfloat16*>(dk);
-  a.dv = static_cast<__nv_bfloat16*>(dv);
+  (void)dk;  // written through tdk and tdv
+  (void)dv;
   a.N = s.N;
   a.Hq = s.Hq;
   a.Hkv = s.Hkv;
@@ -687,7 +710,7 @@ cudaError_t launch_bwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.nk) * a.BHkv;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ctl.ev_after_main && (e = cudaEventRecord(ctl.ev_after_main, stream)) != cudaSuccess) return e;
@@ -707,10 +730,10 @@ size_t bwd_workspace_bytes(const AttnShape& s) {
 }
 
 cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
-                       const float* lse, void* dq, void* dk, void* dv, void* workspace, const LaunchCtl& ctl,
-                       cudaStream_t stream) {
-#define FA_BWD_ARGS s, tq, tk, tv, tdo, o, o_resid, dout, lse, dq, dk, dv, workspace, ctl, stream
+                       const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const void* o,
+                       const void* o_resid, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       void* workspace, const LaunchCtl& ctl, cudaStream_t stream) {
+#define FA_BWD_ARGS s, tq, tk, tv, tdo, tdk, tdv, o, o_resid, dout, lse, dq, dk, dv, workspace, ctl, stream
   switch (s.mask_kind() + (s.d == 64 ? 0 : 3)) {
     case 0: return launch_bwd_t<64, 0>(FA_BWD_ARGS);
     case 1: return launch_bwd_t<64, 1>(FA_BWD_ARGS);

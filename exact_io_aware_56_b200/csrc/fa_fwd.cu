@@ -116,7 +116,8 @@ struct FwdCfg {
   // otherwise the finished Q_t buffer holds them.
   static constexpr bool kOwnStage = !F8 && kTileBytes < 2 * 16384;
   static constexpr int kOffStage = (kOffBar + kBarBytes + 1023) / 1024 * 1024;
-  static constexpr int kSmemBytes = (kOwnStage ? kOffStage + 4 * 16384 : kOffBar + kBarBytes) + 1024;  // + alignment slack
+  // + alignment slack
+  static constexpr int kSmemBytes = (kOwnStage ? kOffStage + 4 * 16384 : kOffBar + kBarBytes) + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(kSmemBytes > 114 * 1024, "one CTA per SM (owns all tensor memory)");

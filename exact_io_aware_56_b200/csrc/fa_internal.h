@@ -76,10 +76,11 @@ cudaError_t launch_quantize_fp8(const void* x, void* codes, float* scales, int B
 
 size_t bwd_workspace_bytes(const AttnShape& s);
 
+// tdk and tdv: bf16 tensor maps of dk and dv laid out like k (128-row boxes).
 cudaError_t launch_bwd(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const void* o, const void* o_resid, const void* dout,
-                       const float* lse, void* dq,
-                       void* dk, void* dv, void* workspace, const LaunchCtl& ctl, cudaStream_t stream);
+                       const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const void* o,
+                       const void* o_resid, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       void* workspace, const LaunchCtl& ctl, cudaStream_t stream);
 
 // Decode / short-query attention: Nq queries per head against an Nk-key
 // cache, queries at the last Nq positions.
