@@ -85,12 +85,17 @@ constexpr float kRescaleLazy = 8.0f;
 constexpr float kF8Rescale = 4.0f;
 constexpr float kF8Offset = 8.0f - kF8Rescale;
 // Of every 32 exponentials of a row, this many are evaluated on the FMA pipe
-// (exp2_poly) and the rest on the exponential unit. Measured on B200 at
-// N = 8192, d = 128: 0 of 32 is fastest (4, 8, 12 cost 3%, 8%, 14%): the
-// softmax warps are bound by instruction issue, not by the exponential unit,
-// so the extra FMA-pipe instructions only add issue slots. FP8 mode likewise
-// (4 of 16: +0.5%, within noise; 8 of 16: -12%).
+// (exp2_poly, exact at integer arguments like the exponential unit) and the
+// rest on the exponential unit. Measured on B200 at N = 8192, d = 128: 0 of
+// 32 is fastest (4, 8, 12 cost 3%, 8%, 14%); there the softmax is one link
+// of a chain with P V and the next S, and the extra FMA-pipe instructions
+// only lengthen it. FP8 mode likewise (4 of 16: +0.5%, within noise; 8 of
+// 16: -12%). At d = 64 the softmax alone sets the pace (S of the next tile
+// is computed while it runs) and its weights need twice the exponential
+// unit's time of the MMAs: 4 of 32 gains 2% (B = 4, H = 16, N = 2048, with
+// and without the causal mask), 8 of 32 loses 4%.
 constexpr int kPolyPer32 = 0;
+constexpr int kPolyPer32D64 = 4;
 
 // F8: e4m3 Q, K, V with block scales (the FP8 mode); otherwise bf16.
 template <int D, bool F8 = false>
@@ -597,8 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               float x0, x1;
               ffma2(x0, x1, __uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1]), sl2,
                     sl2, neg_m, neg_m);
-              const float p0 = (2 * i < kPolyPer32) ? exp2_poly(x0) : ex2(x0);
-              const float p1 = (2 * i + 1 < kPolyPer32) ? exp2_poly(x1) : ex2(x1);
+              constexpr int kPoly = D == 64 ? kPolyPer32D64 : kPolyPer32;
+              const float p0 = (2 * i < kPoly) ? exp2_poly(x0) : ex2(x0);
+              const float p1 = (2 * i + 1 < kPoly) ? exp2_poly(x1) : ex2(x1);
               fadd2(ps[(2 * i) & 7], ps[(2 * i + 1) & 7], ps[(2 * i) & 7], ps[(2 * i + 1) & 7], p0, p1);
               pk[i] = pack_bf16x2(p0, p1);
             }
@@ -607,16 +613,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (h == 0 && rescale) {
           // O holds every earlier product (see the ordering argument above);
-          // scale this row by alpha before P V is added to it (32 columns
-          // per tensor-memory round trip: more would spill at d = 128, where
-          // 64 scores are still live here).
+          // scale this row by alpha before P V is added to it, two columns
+          // per packed multiply. d = 64: one tensor-memory round trip (two
+          // loads, one wait); d = 128: 32 columns per round trip (64 would
+          // spill, with 64 scores still live here).
+          if constexpr (D == 64) {
+            uint32_t oo[64];
+            uint32_t(&o0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oo[0]);
+            uint32_t(&o1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&oo[32]);
+            tmem_ld32_nowait(tO, o0);
+            tmem_ld32_nowait(tO + 32, o1);
+            tmem_ld_wait(o0);
+            tmem_ld_tie(o1);
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o32[32];
-            tmem_ld32(tO + c * 32, o32);
+            for (int i = 0; i < 64; i += 2) {
+              float y0, y1;
+              fmul2(y0, y1, __uint_as_float(oo[i]), __uint_as_float(oo[i + 1]), alpha, alpha);
+              oo[i] = __float_as_uint(y0);
+              oo[i + 1] = __float_as_uint(y1);
+            }
+            tmem_st32(tO, o0);
+            tmem_st32(tO + 32, o1);
+          } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
-            tmem_st32(tO + c * 32, o32);
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o32[32];
+              tmem_ld32(tO + c * 32, o32);
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                float y0, y1;
+                fmul2(y0, y1, __uint_as_float(o32[i]), __uint_as_float(o32[i + 1]), alpha, alpha);
+                o32[i] = __float_as_uint(y0);
+                o32[i + 1] = __float_as_uint(y1);
+              }
+              tmem_st32(tO + c * 32, o32);
+            }
           }
         }
         tmem_st_wait();
