@@ -60,10 +60,12 @@ namespace {
 
 constexpr int kBM = 128;   // query rows per Q tile
 constexpr int kBN = 128;   // keys per K/V tile
-constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8;   // Q and K
-constexpr int kMmaWarp = 9;
-constexpr int kVProducerWarp = 10;  // V
+// One-tile form (d = 64, two CTAs per SM): register shares of the softmax
+// warpgroup and of the producer / MMA warpgroup (setmaxnreg), summing to
+// what a launch at 128 registers per thread gives the CTA.
+constexpr int kSoftmaxRegs1 = 192;
+constexpr int kOtherRegs1 = 64;
+static_assert(kSoftmaxRegs1 + kOtherRegs1 == 2 * 128, "register split of the one-tile form");
 // Rescale threshold (log2 units): a warp rescales its O rows only when some
 // row's running max grew by more than this. With the O residual (the
 // training path, whose backward forms D from O to ~16 bits) it is 0: every
@@ -98,34 +100,53 @@ constexpr int kPolyPer32 = 0;
 constexpr int kPolyPer32D64 = 4;
 
 // F8: e4m3 Q, K, V with block scales (the FP8 mode); otherwise bf16.
-template <int D, bool F8 = false>
+// T: Q tiles per CTA. T = 2 (one CTA per SM, all of its tensor memory) is
+// the general form; T = 1 (d = 64 in bf16 only) runs two CTAs per SM, each
+// with half the tensor memory and shared memory, so that one CTA's start
+// and epilogue overlap the other's key-tile loop.
+template <int D, bool F8 = false, int T = 2>
 struct FwdCfg {
+  static_assert(T == 2 || (T == 1 && D == 64 && !F8), "the one-tile form is the d = 64 bf16 kernel");
+  static constexpr int kThreads = T == 1 ? 256 : 384;
+  static constexpr int kMinBlocks = T == 1 ? 2 : 1;  // CTAs per SM
+  static constexpr int kProducerWarp = 4 * T;        // Q and K
+  static constexpr int kMmaWarp = 4 * T + 1;
+  static constexpr int kVProducerWarp = 4 * T + 2;   // V
   static constexpr int kElem = F8 ? 1 : 2;              // bytes per element
   static constexpr int kBoxCols = 128 / kElem;          // elements per 128-byte swizzle row
   static constexpr int kKStep = 32 / kElem;             // MMA K per instruction (16 bf16, 32 e4m3)
   // K and V rings: K_j is free once both S products of tile j are issued,
   // V_j only after both P V products, so K gets the deeper ring where
   // shared memory is short (d = 128 in bf16: 3 K stages, 2 V stages).
-  static constexpr int kKStages = (D * kElem == 256) ? 3 : 4;
-  static constexpr int kVStages = (D * kElem == 256) ? 2 : 4;
+  static constexpr int kKStages = T == 1 ? 2 : (D * kElem == 256) ? 3 : 4;
+  static constexpr int kVStages = T == 1 ? 2 : (D * kElem == 256) ? 2 : 4;
   static constexpr int kBoxBytes = kBN * 128;           // one 128-byte-wide TMA box of a 128-row tile
   static constexpr int kBoxes = D * kElem / 128;
   static constexpr int kTileBytes = kBoxBytes * kBoxes;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffK = T * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
   static constexpr int kBarBytes = 512;
   // Output staging (the epilogue, bf16 mode): two 16-KB boxes per Q tile.
-  // Where a Q tile is smaller than that (d = 64) they get their own region;
-  // otherwise the finished Q_t buffer holds them.
-  static constexpr bool kOwnStage = !F8 && kTileBytes < 2 * 16384;
+  // At d = 128 the finished Q_t buffer holds them; at d = 64 they get their
+  // own region, except in the one-tile form, whose two boxes are the Q
+  // buffer and one box of its own.
+  static constexpr bool kOwnStage = !F8 && (T == 1 || kTileBytes < 2 * 16384);
   static constexpr int kOffStage = (kOffBar + kBarBytes + 1023) / 1024 * 1024;
+  static constexpr int kStageBytes = T == 1 ? 16384 : 4 * 16384;
   // + alignment slack
-  static constexpr int kSmemBytes = (kOwnStage ? kOffStage + 4 * 16384 : kOffBar + kBarBytes) + 1024;
-  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kSmemBytes = (kOwnStage ? kOffStage + kStageBytes : kOffBar + kBarBytes) + 1024;
+  // Tensor memory: S_t at [128t, 128t + 128), O_t at kColO + D t, P_t (the
+  // separate-P schedule) at kColP + 64t.
+  static constexpr uint32_t kTmemCols = T == 1 ? 256 : 512;
+  static constexpr uint32_t kColO = T == 1 ? 128 : 256;
+  static constexpr uint32_t kColP = T == 1 ? 192 : 384;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert(kSmemBytes > 114 * 1024, "one CTA per SM (owns all tensor memory)");
+  // One CTA per SM (it owns all tensor memory), or exactly two.
+  static_assert(T == 1 ? (kSmemBytes <= 228 * 1024 / 2 - 1024 && 3 * kSmemBytes > 228 * 1024)
+                       : kSmemBytes > 114 * 1024,
+                "CTAs per SM");
 };
 
 // Block scales of the FP8 mode: Q and K per 128-row block of a head
@@ -140,7 +161,8 @@ struct FwdArgs {
   void* o;              // stored through tmO, except in FP8 mode
   const void* o_resid;  // optional: bf16(O - bf16(O)), the rounding residual of o (stored through tmR)
   float* lse;
-  int N, Hq, Hkv, BH, n_pairs, nk;
+  int N, Hq, Hkv, BH, nk;
+  int n_pairs;  // work units per head: pairs of Q tiles (single tiles in the one-tile form)
   int group;  // heads per scheduling group (see the work-unit comment)
   int window;  // left window (a huge value when there is none), mask kind 2
   int prefix;  // prefix length, mask kind 2
@@ -160,7 +182,8 @@ struct FwdBars {
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(FwdBars) <= FwdCfg<64>::kBarBytes, "barrier block exceeds its shared-memory reservation");
+static_assert(sizeof(FwdBars) <= FwdCfg<128>::kBarBytes && sizeof(FwdBars) <= FwdCfg<64, false, 1>::kBarBytes,
+              "barrier block exceeds its shared-memory reservation");
 
 // Key j visible to query i under mask kind 2.
 __device__ __forceinline__ bool visible2(int i, int j, int window, int prefix) {
@@ -169,12 +192,13 @@ __device__ __forceinline__ bool visible2(int i, int j, int window, int prefix) {
 
 // MASK: 0 none, 1 causal, 2 causal with a left window and/or a prefix.
 // F8: e4m3 operands with block scales (FP8 mode, masks 0 and 1).
-template <int D, int MASK, bool F8 = false>
-__global__ void __launch_bounds__(kThreads, 1)
+// T: Q tiles per CTA (see FwdCfg).
+template <int D, int MASK, bool F8 = false, int T = 2>
+__global__ void __launch_bounds__(FwdCfg<D, F8, T>::kThreads, FwdCfg<D, F8, T>::kMinBlocks)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                const __grid_constant__ CUtensorMap tmR, const FwdArgs a) {
-  using C = FwdCfg<D, F8>;
+  using C = FwdCfg<D, F8, T>;
   static_assert(!F8 || MASK != 2, "FP8 mode covers the unmasked and causal forward");
   // Separate-P schedule: with d = 64 tensor memory has room for P next to S
   // (S_t at [128t, 128t+128), O_t at [256 + 64t, ...), P_t at [384 + 64t,
@@ -194,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work unit: (batch*head, pair of Q tiles). Heads are taken in groups
+  // Work unit: (batch*head, T consecutive Q tiles: a pair, or one tile in the
+  // one-tile form). Heads are taken in groups
   // (all heads in one group when causal, where longest-first order matters
   // most; otherwise small enough that a group's K/V tiles stay in L2 while
   // the resident CTAs stream them); within a group the heaviest pairs
@@ -209,14 +234,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = bh % a.Hq;
   const int b = bh / a.Hq;
   const int kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
-  const int q0 = pair * 2 * kBM;
+  const int q0 = pair * T * kBM;
   int n_t[2];
   // Mask kind 2: both Q tiles walk one K/V stream, the prefix tiles [0, pre)
   // then the window tiles [win0, win1): stream position u holds key tile
   // u < pre ? u : win0 + (u - pre). Tiles in the gap are never visited.
   int pre = 0, win0 = 0;
   if (MASK == 2) {
-    const int q_hi = min(q0 + 2 * kBM, a.N) - 1;   // highest real query of the pair
+    const int q_hi = min(q0 + T * kBM, a.N) - 1;   // highest real query of the unit
     pre = min(a.nk, (a.prefix + kBN - 1) / kBN);
     const int lo_key = (a.window >= q0) ? 0 : q0 - a.window;
     win0 = max(pre, lo_key / kBN);
@@ -224,8 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     n_t[0] = n_t[1] = pre + max(0, win1 - win0);
   } else {
 #pragma unroll
-    for (int t = 0; t < 2; ++t) n_t[t] = MASK == 1 ? min(a.nk, 2 * pair + t + 1) : a.nk;
+    for (int t = 0; t < 2; ++t) n_t[t] = MASK == 1 ? min(a.nk, T * pair + min(t, T - 1) + 1) : a.nk;
   }
+  // n_t[1] is the unit's K/V stream length (n_t[0] in the one-tile form).
   auto key_tile = [&](int u) { return (MASK == 2 && u >= pre) ? win0 + (u - pre) : u; };
 
   if (threadIdx.x == 0) {
@@ -252,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == C::kMmaWarp) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
@@ -266,160 +292,210 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------- Q, K producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      int k_last[KS];
-#pragma unroll
-      for (int s = 0; s < KS; ++s) k_last[s] = -1;
-      mbar_arrive_expect_tx(&bars->q_full, 2 * C::kTileBytes);
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(&tmQ, &bars->q_full, smem + C::kOffQ + t * C::kTileBytes + x * C::kBoxBytes,
-                      x * C::kBoxCols, q0 + t * kBM, bh);
-      const int n = n_t[1];
-      for (int j = 0; j < n; ++j) {
-        const int s = j % KS;
-        const int u = j / KS;
-        if (j >= KS && !wait_bar(&bars->k_empty[s], (u - 1) & 1, w)) break;
-        if (a.ctl.fault == 1 && j == 0) continue;  // test hook: K_0 never arrives
-        mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
-#pragma unroll
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes,
-                      x * C::kBoxCols, key_tile(j) * kBN, kvh);
-        k_last[s] = u;
-      }
-      // Every copy issued must land before the CTA may exit.
-      drain_bar(&bars->q_full, 0, w);
-#pragma unroll
-      for (int s = 0; s < KS; ++s)
-        if (k_last[s] >= 0) drain_bar(&bars->k_full[s], k_last[s] & 1, w);
-    }
-  } else if (warp == kVProducerWarp) {
-    // ----------------------------------------------------------- V producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmV);
-      int v_last[VS];
-#pragma unroll
-      for (int s = 0; s < VS; ++s) v_last[s] = -1;
-      const int n = n_t[1];
-      for (int j = 0; j < n; ++j) {
-        const int s = j % VS;
-        const int u = j / VS;
-        if (j >= VS && !wait_bar(&bars->v_empty[s], (u - 1) & 1, w)) break;
-        mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
-#pragma unroll
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes,
-                      x * C::kBoxCols, key_tile(j) * kBN, kvh);
-        v_last[s] = u;
-      }
-#pragma unroll
-      for (int s = 0; s < VS; ++s)
-        if (v_last[s] >= 0) drain_bar(&bars->v_full[s], v_last[s] & 1, w);
-    }
-  } else if (warp == kMmaWarp) {
-    // ----------------------------------------------------------- MMA issue
-    // The whole warp runs this loop (descriptors stay warp-uniform); the
-    // elected lane issues the tcgen05 instructions.
-    const bool leader = elect_one();
-    auto all = [](bool b) { return __all_sync(0xffffffffu, b); };
-    {
-      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(kBM, kBN, false, false) : idesc_bf16(kBM, kBN, false, false);
-      constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(kBM, D, false, true) : idesc_bf16(kBM, D, false, true);
-      constexpr int KSTEP = C::kKStep;  // MMA K per instruction (16 bf16, 32 e4m3)
-      const uint32_t tS[2] = {tmem, tmem + 128u};
-      // A operand (P) of O += P V: over S, or in its own columns (SEP).
-      const uint32_t tP[2] = {SEP ? tmem + 384u : tmem, SEP ? tmem + 448u : tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
-      // Operand descriptors computed once and stepped by byte offsets
-      // (sdesc_step): K step k of a K-major tile is 32 bytes within a
-      // 128-byte swizzle row, boxes kBoxBytes apart; of the MN-major V tile,
-      // KSTEP rows of 128 bytes.
-      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
-      const uint64_t dV = sdesc_sw128(sV, C::kBoxBytes, 1024);
-      auto ofs_kmaj = [](int k) { return static_cast<uint32_t>((k / 4) * C::kBoxBytes + (k % 4) * 32); };
-      auto issue_s = [&](int t, int j) {
-        const uint64_t qa = sdesc_step(dQ, t * C::kTileBytes);
-        const uint64_t ka = sdesc_step(dK, (j % KS) * C::kTileBytes);
-        if constexpr (F8) {
-          // Each K step is 32 bytes of a 128-byte swizzle row (32 e4m3).
-#pragma unroll
-          for (int k = 0; k < D / KSTEP; ++k)
-            mma_ss_f8(tS[t], sdesc_step(qa, ofs_kmaj(k)), sdesc_step(ka, ofs_kmaj(k)), idesc_qk, k > 0, leader);
-        } else {
-#pragma unroll
-          for (int k = 0; k < D / KSTEP; k += 4)
-            mma_ss_x4(tS[t], sdesc_step(qa, ofs_kmaj(k)), sdesc_step(qa, ofs_kmaj(k + 1)),
-                      sdesc_step(qa, ofs_kmaj(k + 2)), sdesc_step(qa, ofs_kmaj(k + 3)), sdesc_step(ka, ofs_kmaj(k)),
-                      sdesc_step(ka, ofs_kmaj(k + 1)), sdesc_step(ka, ofs_kmaj(k + 2)),
-                      sdesc_step(ka, ofs_kmaj(k + 3)), idesc_qk, k > 0, leader);
+  if (warp >= 4 * T) {
+    // Producers and the MMA warp (one-tile form: the smaller register share).
+    if constexpr (T == 1) regs_dec<kOtherRegs1>();
+    if (warp == C::kProducerWarp) {
+      // ------------------------------------------------------- Q, K producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        int k_last[KS];
+    #pragma unroll
+        for (int s = 0; s < KS; ++s) k_last[s] = -1;
+        mbar_arrive_expect_tx(&bars->q_full, T * C::kTileBytes);
+    #pragma unroll
+        for (int t = 0; t < T; ++t)
+    #pragma unroll
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_3d(&tmQ, &bars->q_full, smem + C::kOffQ + t * C::kTileBytes + x * C::kBoxBytes,
+                        x * C::kBoxCols, q0 + t * kBM, bh);
+        const int n = n_t[1];
+        for (int j = 0; j < n; ++j) {
+          const int s = j % KS;
+          const int u = j / KS;
+          if (j >= KS && !wait_bar(&bars->k_empty[s], (u - 1) & 1, w)) break;
+          if (a.ctl.fault == 1 && j == 0) continue;  // test hook: K_0 never arrives
+          mbar_arrive_expect_tx(&bars->k_full[s], C::kTileBytes);
+    #pragma unroll
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_3d(&tmK, &bars->k_full[s], smem + C::kOffK + s * C::kTileBytes + x * C::kBoxBytes,
+                        x * C::kBoxCols, key_tile(j) * kBN, kvh);
+          k_last[s] = u;
         }
-        mma_commit(&bars->s_full[t], leader);
-      };
-      // Half h of P V: keys [64h, 64h + 64).
-      auto issue_pv = [&](int t, int j, int h) {
-        const uint64_t va = sdesc_step(dV, (j % VS) * C::kTileBytes);
-        // P: KSTEP keys per step = 8 tensor-memory columns (bf16 pairs or e4m3
-        // quads); V: KSTEP key rows of 128 bytes (MN-major).
-        constexpr int KH = kBN / KSTEP / 2;
-        if constexpr (F8) {
-#pragma unroll
-          for (int k = h * KH; k < h * KH + KH; ++k)
-            mma_ts_f8(tO[t], tP[t] + k * 8, sdesc_step(va, k * KSTEP * 128), idesc_pv, (j > 0 || k > 0) ? 1u : 0u,
-                      leader);
-        } else {
-          static_assert(F8 || KH == 4, "one group of four MMAs per half");
-          const int k = h * KH;
-          mma_ts_x4(tO[t], tP[t] + k * 8, tP[t] + (k + 1) * 8, tP[t] + (k + 2) * 8, tP[t] + (k + 3) * 8,
-                    sdesc_step(va, k * KSTEP * 128), sdesc_step(va, (k + 1) * KSTEP * 128),
-                    sdesc_step(va, (k + 2) * KSTEP * 128), sdesc_step(va, (k + 3) * KSTEP * 128), idesc_pv,
-                    (j > 0 || k > 0) ? 1u : 0u, leader);
-        }
-      };
-      const int n0 = n_t[0], n1 = n_t[1];
-      bool ok = all(wait_bar(&bars->q_full, 0, w)) && all(wait_bar(&bars->k_full[0], 0, w));
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        mma_commit(&bars->k_empty[0], leader);  // K_0 read by both S products
+        // Every copy issued must land before the CTA may exit.
+        drain_bar(&bars->q_full, 0, w);
+    #pragma unroll
+        for (int s = 0; s < KS; ++s)
+          if (k_last[s] >= 0) drain_bar(&bars->k_full[s], k_last[s] & 1, w);
       }
-      for (int j = 0; ok && j < n1; ++j) {
-        const int s = j % VS;                   // V_j stage
-        const uint32_t par = (j / VS) & 1;
-        const int jn = j + 1;
-        if constexpr (SEP) {
-          // S_t of tile j + 1 as soon as the softmax has loaded S_t of tile
-          // j; then this tile's P V. pv_done tells the softmax when P_t and
-          // O_t may be written again.
-          if (j < n0) {
-            if (jn < n0) {
-              if (!(ok = all(wait_bar(&bars->s_free[0], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
+    } else if (warp == C::kVProducerWarp) {
+      // ----------------------------------------------------------- V producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmV);
+        int v_last[VS];
+    #pragma unroll
+        for (int s = 0; s < VS; ++s) v_last[s] = -1;
+        const int n = n_t[1];
+        for (int j = 0; j < n; ++j) {
+          const int s = j % VS;
+          const int u = j / VS;
+          if (j >= VS && !wait_bar(&bars->v_empty[s], (u - 1) & 1, w)) break;
+          mbar_arrive_expect_tx(&bars->v_full[s], C::kTileBytes);
+    #pragma unroll
+          for (int x = 0; x < C::kBoxes; ++x)
+            tma_load_3d(&tmV, &bars->v_full[s], smem + C::kOffV + s * C::kTileBytes + x * C::kBoxBytes,
+                        x * C::kBoxCols, key_tile(j) * kBN, kvh);
+          v_last[s] = u;
+        }
+    #pragma unroll
+        for (int s = 0; s < VS; ++s)
+          if (v_last[s] >= 0) drain_bar(&bars->v_full[s], v_last[s] & 1, w);
+      }
+    } else if (warp == C::kMmaWarp) {
+      // ----------------------------------------------------------- MMA issue
+      // The whole warp runs this loop (descriptors stay warp-uniform); the
+      // elected lane issues the tcgen05 instructions.
+      const bool leader = elect_one();
+      auto all = [](bool b) { return __all_sync(0xffffffffu, b); };
+      {
+        constexpr uint32_t idesc_qk = F8 ? idesc_e4m3(kBM, kBN, false, false) : idesc_bf16(kBM, kBN, false, false);
+        constexpr uint32_t idesc_pv = F8 ? idesc_e4m3(kBM, D, false, true) : idesc_bf16(kBM, D, false, true);
+        constexpr int KSTEP = C::kKStep;  // MMA K per instruction (16 bf16, 32 e4m3)
+        const uint32_t tS[2] = {tmem, tmem + 128u};
+        // A operand (P) of O += P V: over S, or in its own columns (SEP).
+        const uint32_t tP[2] = {SEP ? tmem + C::kColP : tmem, SEP ? tmem + C::kColP + 64u : tmem + 128u};
+        const uint32_t tO[2] = {tmem + C::kColO, tmem + C::kColO + D};
+        // Operand descriptors computed once and stepped by byte offsets
+        // (sdesc_step): K step k of a K-major tile is 32 bytes within a
+        // 128-byte swizzle row, boxes kBoxBytes apart; of the MN-major V tile,
+        // KSTEP rows of 128 bytes.
+        const uint64_t dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
+        const uint64_t dV = sdesc_sw128(sV, C::kBoxBytes, 1024);
+        auto ofs_kmaj = [](int k) { return static_cast<uint32_t>((k / 4) * C::kBoxBytes + (k % 4) * 32); };
+        auto issue_s = [&](int t, int j) {
+          const uint64_t qa = sdesc_step(dQ, t * C::kTileBytes);
+          const uint64_t ka = sdesc_step(dK, (j % KS) * C::kTileBytes);
+          if constexpr (F8) {
+            // Each K step is 32 bytes of a 128-byte swizzle row (32 e4m3).
+    #pragma unroll
+            for (int k = 0; k < D / KSTEP; ++k)
+              mma_ss_f8(tS[t], sdesc_step(qa, ofs_kmaj(k)), sdesc_step(ka, ofs_kmaj(k)), idesc_qk, k > 0, leader);
+          } else {
+    #pragma unroll
+            for (int k = 0; k < D / KSTEP; k += 4)
+              mma_ss_x4(tS[t], sdesc_step(qa, ofs_kmaj(k)), sdesc_step(qa, ofs_kmaj(k + 1)),
+                        sdesc_step(qa, ofs_kmaj(k + 2)), sdesc_step(qa, ofs_kmaj(k + 3)), sdesc_step(ka, ofs_kmaj(k)),
+                        sdesc_step(ka, ofs_kmaj(k + 1)), sdesc_step(ka, ofs_kmaj(k + 2)),
+                        sdesc_step(ka, ofs_kmaj(k + 3)), idesc_qk, k > 0, leader);
+          }
+          mma_commit(&bars->s_full[t], leader);
+        };
+        // Half h of P V: keys [64h, 64h + 64).
+        auto issue_pv = [&](int t, int j, int h) {
+          const uint64_t va = sdesc_step(dV, (j % VS) * C::kTileBytes);
+          // P: KSTEP keys per step = 8 tensor-memory columns (bf16 pairs or e4m3
+          // quads); V: KSTEP key rows of 128 bytes (MN-major).
+          constexpr int KH = kBN / KSTEP / 2;
+          if constexpr (F8) {
+    #pragma unroll
+            for (int k = h * KH; k < h * KH + KH; ++k)
+              mma_ts_f8(tO[t], tP[t] + k * 8, sdesc_step(va, k * KSTEP * 128), idesc_pv, (j > 0 || k > 0) ? 1u : 0u,
+                        leader);
+          } else {
+            static_assert(F8 || KH == 4, "one group of four MMAs per half");
+            const int k = h * KH;
+            mma_ts_x4(tO[t], tP[t] + k * 8, tP[t] + (k + 1) * 8, tP[t] + (k + 2) * 8, tP[t] + (k + 3) * 8,
+                      sdesc_step(va, k * KSTEP * 128), sdesc_step(va, (k + 1) * KSTEP * 128),
+                      sdesc_step(va, (k + 2) * KSTEP * 128), sdesc_step(va, (k + 3) * KSTEP * 128), idesc_pv,
+                      (j > 0 || k > 0) ? 1u : 0u, leader);
+          }
+        };
+        const int n0 = n_t[0], n1 = n_t[1];
+        bool ok = all(wait_bar(&bars->q_full, 0, w)) && all(wait_bar(&bars->k_full[0], 0, w));
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          if constexpr (T == 2) issue_s(1, 0);
+          mma_commit(&bars->k_empty[0], leader);  // K_0 read by the S products
+        }
+        // One-tile form (separate P): S of the next key tile once the softmax
+        // has loaded this one, then this tile's P V.
+        for (int j = 0; T == 1 && ok && j < n0; ++j) {
+          const int s = j % VS;
+          const uint32_t par = (j / VS) & 1;
+          const int jn = j + 1;
+          if (jn < n0) {
+            if (!(ok = all(wait_bar(&bars->s_free[0], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
+              break;
+            tc_fence_after();
+            issue_s(0, jn);
+            mma_commit(&bars->k_empty[jn % KS], leader);
+          }
+          if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
+          tc_fence_after();
+          issue_pv(0, j, 0);
+          if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
+          tc_fence_after();
+          issue_pv(0, j, 1);
+          mma_commit(&bars->pv_done[0], leader);
+          mma_commit(&bars->v_empty[s], leader);
+          if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
+        }
+        for (int j = 0; T == 2 && ok && j < n1; ++j) {
+          const int s = j % VS;                   // V_j stage
+          const uint32_t par = (j / VS) & 1;
+          const int jn = j + 1;
+          if constexpr (SEP) {
+            // S_t of tile j + 1 as soon as the softmax has loaded S_t of tile
+            // j; then this tile's P V. pv_done tells the softmax when P_t and
+            // O_t may be written again.
+            if (j < n0) {
+              if (jn < n0) {
+                if (!(ok = all(wait_bar(&bars->s_free[0], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
+                  break;
+                tc_fence_after();
+                issue_s(0, jn);
+              }
+              if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
+              tc_fence_after();
+              issue_pv(0, j, 0);
+              if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
+              tc_fence_after();
+              issue_pv(0, j, 1);
+              mma_commit(&bars->pv_done[0], leader);
+              if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
+            }
+            if (jn < n1) {
+              if (!(ok = all(wait_bar(&bars->s_free[1], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
                 break;
               tc_fence_after();
-              issue_s(0, jn);
+              issue_s(1, jn);
+              mma_commit(&bars->k_empty[jn % KS], leader);
             }
+            if (!(ok = all(wait_bar(&bars->p_ready[1][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
+            tc_fence_after();
+            issue_pv(1, j, 0);
+            if (!(ok = all(wait_bar(&bars->p_ready[1][1], j & 1, w)))) break;
+            tc_fence_after();
+            issue_pv(1, j, 1);
+            mma_commit(&bars->pv_done[1], leader);
+            mma_commit(&bars->v_empty[s], leader);
+            if (j == n1 - 1) mma_commit(&bars->o_final[1], leader);
+            continue;
+          }
+          if (j < n0) {
             if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
             tc_fence_after();
             issue_pv(0, j, 0);
             if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
             tc_fence_after();
             issue_pv(0, j, 1);
-            mma_commit(&bars->pv_done[0], leader);
             if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
-          }
-          if (jn < n1) {
-            if (!(ok = all(wait_bar(&bars->s_free[1], j & 1, w)) && all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w))))
-              break;
-            tc_fence_after();
-            issue_s(1, jn);
-            mma_commit(&bars->k_empty[jn % KS], leader);
+            if (jn < n0) {
+              if (!(ok = all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w)))) break;
+              issue_s(0, jn);
+            }
           }
           if (!(ok = all(wait_bar(&bars->p_ready[1][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
           tc_fence_after();
@@ -427,43 +503,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = all(wait_bar(&bars->p_ready[1][1], j & 1, w)))) break;
           tc_fence_after();
           issue_pv(1, j, 1);
-          mma_commit(&bars->pv_done[1], leader);
           mma_commit(&bars->v_empty[s], leader);
           if (j == n1 - 1) mma_commit(&bars->o_final[1], leader);
-          continue;
-        }
-        if (j < n0) {
-          if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
-          tc_fence_after();
-          issue_pv(0, j, 0);
-          if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
-          tc_fence_after();
-          issue_pv(0, j, 1);
-          if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
-          if (jn < n0) {
+          if (jn < n1) {
             if (!(ok = all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w)))) break;
-            issue_s(0, jn);
+            issue_s(1, jn);
+            mma_commit(&bars->k_empty[jn % KS], leader);
           }
         }
-        if (!(ok = all(wait_bar(&bars->p_ready[1][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
-        tc_fence_after();
-        issue_pv(1, j, 0);
-        if (!(ok = all(wait_bar(&bars->p_ready[1][1], j & 1, w)))) break;
-        tc_fence_after();
-        issue_pv(1, j, 1);
-        mma_commit(&bars->v_empty[s], leader);
-        if (j == n1 - 1) mma_commit(&bars->o_final[1], leader);
-        if (jn < n1) {
-          if (!(ok = all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w)))) break;
-          issue_s(1, jn);
-          mma_commit(&bars->k_empty[jn % KS], leader);
-        }
+        // All MMAs issued by this thread must finish before tensor memory is freed.
+        mma_commit(&bars->drain, leader);
+        all(drain_bar(&bars->drain, 0, w));
       }
-      // All MMAs issued by this thread must finish before tensor memory is freed.
-      mma_commit(&bars->drain, leader);
-      all(drain_bar(&bars->drain, 0, w));
     }
-  } else if (warp < 8) {
+  } else {
+    if constexpr (T == 1) regs_inc<kSoftmaxRegs1>();
     // ------------------------------------------------------------- softmax
     const int t = warp >> 2;                   // Q tile of this warpgroup
     const int quad = warp & 3;                 // tensor-memory lane quadrant
@@ -471,8 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q0 + t * kBM + r;          // query position
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128u;
-    const uint32_t tPw = SEP ? tmem + lane_off + 384u + t * 64u : tS;  // where this tile's P goes
-    const uint32_t tO = tmem + lane_off + 256u + t * D;
+    const uint32_t tPw = SEP ? tmem + lane_off + C::kColP + t * 64u : tS;  // where this tile's P goes
+    const uint32_t tO = tmem + lane_off + C::kColO + t * D;
     const int n = n_t[t];
     // FP8 mode: the scores come out of the MMA in units of sq * sk (the Q
     // tile's and the K tile's block scales); both fold into the exponent's
@@ -492,7 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[kBN];
-      tmem_ld128(tS, sr);
+      // (With the register split, no instruction may name more than 64
+      // destination registers.)
+      if constexpr (T == 1)
+        tmem_ld64x2(tS, sr);
+      else
+        tmem_ld128(tS, sr);
       if constexpr (SEP) {
         // S_t is in registers: the MMA thread may compute the next tile's S_t.
         tc_fence_before();
@@ -675,12 +734,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kBoxesO = D / 64;  // bf16 output boxes
         constexpr int kSlots = 2;        // 16-KB boxes staged at a time
         const int jobs = qt0 < a.N ? kBoxesO * (a.o_resid ? 2 : 1) : 0;
-        uint8_t* stage = C::kOwnStage ? smem + C::kOffStage + t * 2 * 16384 : smem + C::kOffQ + t * C::kTileBytes;
+        // Box i of this tile stages in slot i % 2: two boxes of the own region
+        // or of the Q_t buffer; in the one-tile form the Q buffer, then the
+        // own box.
+        uint8_t* const slots[2] = {
+            T == 1 ? smem + C::kOffQ : (C::kOwnStage ? smem + C::kOffStage + t * 2 * 16384 : smem + C::kOffQ + t * C::kTileBytes),
+            T == 1 ? smem + C::kOffStage
+                   : (C::kOwnStage ? smem + C::kOffStage + t * 2 * 16384 : smem + C::kOffQ + t * C::kTileBytes) + 16384};
         const bool issuer = r == 0;
         for (int i = 0; i < jobs; ++i) {
           const int x = i % kBoxesO;
           const bool resid = i >= kBoxesO;
-          uint8_t* slot = stage + (i % kSlots) * 16384;
+          uint8_t* slot = slots[i % kSlots];
           // The slot's previous box must have been read by its copy.
           if (i >= kSlots && !(ok = __all_sync(0xffffffffu, wait_bar(&bars->epi_free[t], (i - kSlots) & 1, w)))) break;
           uint32_t oo[64];
@@ -747,22 +812,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == C::kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
-template <int D, int MASK, bool F8 = false>
+// d = 64 in bf16 takes the one-tile form (two CTAs per SM).
+template <int D, int MASK, bool F8 = false, int T = (D == 64 && !F8) ? 1 : 2>
 cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& to, const CUtensorMap& tr, void* o, void* o_resid, float* lse,
                          const LaunchCtl& ctl, cudaStream_t stream,
                          Fp8Scales f8 = Fp8Scales{nullptr, nullptr, nullptr}) {
-  using C = FwdCfg<D, F8>;
-  auto kern = fwd_kernel<D, MASK, F8>;
+  using C = FwdCfg<D, F8, T>;
+  auto kern = fwd_kernel<D, MASK, F8, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  if constexpr (T == 1) {
+    // The register split (setmaxnreg) hands out exactly what a launch at 128
+    // registers per thread gives the CTA; with any other count the softmax
+    // warps' increase could never be granted.
+    static const int launch_regs = [&] {
+      cudaFuncAttributes at{};
+      return cudaFuncGetAttributes(&at, kern) == cudaSuccess ? at.numRegs : -1;
+    }();
+    if (launch_regs != 128) return cudaErrorLaunchOutOfResources;
+  }
   FwdArgs a;
   a.o = o;
   a.o_resid = o_resid;
@@ -772,7 +848,7 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.Hkv = s.Hkv;
   a.BH = s.B * s.Hq;
   a.nk = (s.N + kBN - 1) / kBN;
-  a.n_pairs = (s.N + 2 * kBM - 1) / (2 * kBM);
+  a.n_pairs = (s.N + T * kBM - 1) / (T * kBM);  // units per head
   // Causal units differ in length: keep strict longest-first order over all
   // heads. Non-causal units are equal: group heads for L2 locality.
   a.group = MASK == 1 ? a.BH
@@ -785,7 +861,7 @@ cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtens
   a.ctl = ctl;
   const long long grid = static_cast<long long>(a.n_pairs) * a.BH;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, tr, a);
+  kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, tr, a);
   return cudaGetLastError();
 }
 
