@@ -94,19 +94,23 @@ constexpr float kF8Offset = 8.0f - kF8Rescale;
 // only lengthen it. FP8 mode likewise (4 of 16: +0.5%, within noise; 8 of
 // 16: -12%). At d = 64 the softmax alone sets the pace (S of the next tile
 // is computed while it runs) and its weights need twice the exponential
-// unit's time of the MMAs: 4 of 32 gains 2% (B = 4, H = 16, N = 2048, with
-// and without the causal mask), 8 of 32 loses 4%.
+// unit's time of the MMAs. With two one-tile CTAs per SM (B = 4, H = 16,
+// N = 2048): 4 of 32 gains 2 to 4% without a mask and loses 2.5% causal
+// (0 fastest there), 8 of 32 loses 4 to 7%.
 constexpr int kPolyPer32 = 0;
-constexpr int kPolyPer32D64 = 4;
+template <int D, int MASK>
+constexpr int poly_per32() {
+  return (D == 64 && MASK == 0) ? 4 : kPolyPer32;
+}
 
 // F8: e4m3 Q, K, V with block scales (the FP8 mode); otherwise bf16.
 // T: Q tiles per CTA. T = 2 (one CTA per SM, all of its tensor memory) is
-// the general form; T = 1 (d = 64 in bf16 only) runs two CTAs per SM, each
-// with half the tensor memory and shared memory, so that one CTA's start
-// and epilogue overlap the other's key-tile loop.
+// the general form; T = 1 (d = 64 in bf16, and the FP8 mode: 128-byte rows)
+// runs two CTAs per SM, each with half the tensor memory and shared memory,
+// so that one CTA's start and epilogue overlap the other's key-tile loop.
 template <int D, bool F8 = false, int T = 2>
 struct FwdCfg {
-  static_assert(T == 2 || (T == 1 && D == 64 && !F8), "the one-tile form is the d = 64 bf16 kernel");
+  static_assert(T == 2 || (T == 1 && D * (F8 ? 1 : 2) == 128), "the one-tile form takes 128-byte rows (d = 64 bf16, FP8)");
   static constexpr int kThreads = T == 1 ? 256 : 384;
   static constexpr int kMinBlocks = T == 1 ? 2 : 1;  // CTAs per SM
   static constexpr int kProducerWarp = 4 * T;        // Q and K
@@ -419,9 +423,29 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, T>::kThreads, FwdCfg<D, F8, T>::
           if constexpr (T == 2) issue_s(1, 0);
           mma_commit(&bars->k_empty[0], leader);  // K_0 read by the S products
         }
-        // One-tile form (separate P): S of the next key tile once the softmax
-        // has loaded this one, then this tile's P V.
-        for (int j = 0; T == 1 && ok && j < n0; ++j) {
+        // One-tile form, P over S (FP8): this tile's P V, then S of the next
+        // key tile over the P it has consumed.
+        for (int j = 0; T == 1 && !SEP && ok && j < n0; ++j) {
+          const int s = j % VS;
+          const uint32_t par = (j / VS) & 1;
+          const int jn = j + 1;
+          if (!(ok = all(wait_bar(&bars->p_ready[0][0], j & 1, w)) && all(wait_bar(&bars->v_full[s], par, w)))) break;
+          tc_fence_after();
+          issue_pv(0, j, 0);
+          if (!(ok = all(wait_bar(&bars->p_ready[0][1], j & 1, w)))) break;
+          tc_fence_after();
+          issue_pv(0, j, 1);
+          mma_commit(&bars->v_empty[s], leader);
+          if (j == n0 - 1) mma_commit(&bars->o_final[0], leader);
+          if (jn < n0) {
+            if (!(ok = all(wait_bar(&bars->k_full[jn % KS], (jn / KS) & 1, w)))) break;
+            issue_s(0, jn);
+            mma_commit(&bars->k_empty[jn % KS], leader);
+          }
+        }
+        // One-tile form, separate P (d = 64): S of the next key tile once the
+        // softmax has loaded this one, then this tile's P V.
+        for (int j = 0; T == 1 && SEP && ok && j < n0; ++j) {
           const int s = j % VS;
           const uint32_t par = (j / VS) & 1;
           const int jn = j + 1;
@@ -661,7 +685,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, T>::kThreads, FwdCfg<D, F8, T>::
               float x0, x1;
               ffma2(x0, x1, __uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1]), sl2,
                     sl2, neg_m, neg_m);
-              constexpr int kPoly = D == 64 ? kPolyPer32D64 : kPolyPer32;
+              constexpr int kPoly = poly_per32<D, MASK>();
               const float p0 = (2 * i < kPoly) ? exp2_poly(x0) : ex2(x0);
               const float p1 = (2 * i + 1 < kPoly) ? exp2_poly(x1) : ex2(x1);
               fadd2(ps[(2 * i) & 7], ps[(2 * i + 1) & 7], ps[(2 * i) & 7], ps[(2 * i + 1) & 7], p0, p1);
@@ -819,8 +843,9 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, T>::kThreads, FwdCfg<D, F8, T>::
   }
 }
 
-// d = 64 in bf16 takes the one-tile form (two CTAs per SM).
-template <int D, int MASK, bool F8 = false, int T = (D == 64 && !F8) ? 1 : 2>
+// 128-byte rows (d = 64 in bf16, the FP8 mode) take the one-tile form (two
+// CTAs per SM).
+template <int D, int MASK, bool F8 = false, int T = (D * (F8 ? 1 : 2) == 128) ? 1 : 2>
 cudaError_t launch_fwd_t(const AttnShape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& to, const CUtensorMap& tr, void* o, void* o_resid, float* lse,
                          const LaunchCtl& ctl, cudaStream_t stream,
