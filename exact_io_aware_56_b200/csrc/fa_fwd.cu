@@ -92,8 +92,9 @@ constexpr float kF8Offset = 8.0f - kF8Rescale;
 // 32 is fastest (4, 8, 12 cost 3%, 8%, 14%); there the softmax is one link
 // of a chain with P V and the next S, and the extra FMA-pipe instructions
 // only lengthen it. FP8 mode, one-tile form (B = 2, H = 16, N = 8192 and
-// the 16384-token GQA shape): 2 of every 16 is fastest (+3.5% and +5.5%
-// against none; 4 of 16 +1.5% and +2.5%, 6 of 16 -5%, 8 of 16 -12%). At d = 64 the softmax alone sets the pace (S of the next tile
+// the 16384-token GQA shape): 2 of every 16 is fastest (+1.6% and +2.9%
+// against 4 of 16, which had gained 0.6 to 2.4% against none; 6 of 16:
+// -6%; 8 of 16: -12%). At d = 64 the softmax alone sets the pace (S of the next tile
 // is computed while it runs) and its weights need twice the exponential
 // unit's time of the MMAs. With two one-tile CTAs per SM (B = 4, H = 16,
 // N = 2048): 4 of 32 gains 2 to 4% without a mask and loses 2.5% causal
