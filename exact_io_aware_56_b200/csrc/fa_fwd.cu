@@ -88,22 +88,24 @@ constexpr float kF8Rescale = 4.0f;
 constexpr float kF8Offset = 8.0f - kF8Rescale;
 // Of every 32 exponentials of a row, this many are evaluated on the FMA pipe
 // (exp2_poly, exact at integer arguments like the exponential unit) and the
-// rest on the exponential unit. Measured on B200 at N = 8192, d = 128: 0 of
-// 32 is fastest (4, 8, 12 cost 3%, 8%, 14%); there the softmax is one link
-// of a chain with P V and the next S, and the extra FMA-pipe instructions
-// only lengthen it. FP8 mode, one-tile form (B = 2, H = 16, N = 8192 and
-// the 16384-token GQA shape): 2 of every 16 is fastest (+1.6% and +2.9%
+// rest on the exponential unit. At d = 128 the softmax is one link of a
+// chain with P V and the next S, so FMA-pipe instructions mostly lengthen
+// it: measured on B200 at N = 8192, 4, 8, 12 of 32 cost 3%, 8%, 14% (with
+// per-row epilogue stores and default waits); with the current kernel 2 of
+// 32 gains ~1% at 8192 tokens and 1-4% on the 16384-token GQA forward, 1 of
+// 32 nothing. FP8 mode, one-tile form (B = 2, H = 16, N = 8192 and the
+// 16384-token GQA shape): 2 of every 16 is fastest (+1.6% and +2.9%
 // against 4 of 16, which had gained 0.6 to 2.4% against none; 6 of 16:
-// -6%; 8 of 16: -12%). At d = 64 the softmax alone sets the pace (S of the next tile
-// is computed while it runs) and its weights need twice the exponential
-// unit's time of the MMAs. With two one-tile CTAs per SM (B = 4, H = 16,
-// N = 2048): 4 of 32 gains 2 to 4% without a mask and loses 2.5% causal
-// (0 fastest there), 8 of 32 loses 4 to 7%.
-constexpr int kPolyPer32 = 0;
+// -6%; 8 of 16: -12%). At d = 64 the softmax alone sets the pace (S of the
+// next tile is computed while it runs) and its weights need twice the
+// exponential unit's time of the MMAs. With two one-tile CTAs per SM
+// (B = 4, H = 16, N = 2048): 4 of 32 gains 2 to 4% without a mask and
+// loses 2.5% causal (0 fastest there; 2 of 32 -0.6%), 8 of 32 loses 4 to 7%.
+constexpr int kPolyPer32 = 2;
 constexpr int kPolyPer16F8 = 2;
 template <int D, int MASK>
 constexpr int poly_per32() {
-  return (D == 64 && MASK == 0) ? 4 : kPolyPer32;
+  return D == 64 ? (MASK == 0 ? 4 : 0) : kPolyPer32;
 }
 
 // F8: e4m3 Q, K, V with block scales (the FP8 mode); otherwise bf16.
