@@ -93,16 +93,17 @@ constexpr float kF8Offset = 8.0f - kF8Rescale;
 // it: measured on B200 at N = 8192, 4, 8, 12 of 32 cost 3%, 8%, 14% (with
 // per-row epilogue stores and default waits); with the current kernel 2 of
 // 32 gains ~1% at 8192 tokens and 1-4% on the 16384-token GQA forward, 1 of
-// 32 nothing. FP8 mode, one-tile form (B = 2, H = 16, N = 8192 and the
-// 16384-token GQA shape): 2 of every 16 is fastest (+1.6% and +2.9%
-// against 4 of 16, which had gained 0.6 to 2.4% against none; 6 of 16:
-// -6%; 8 of 16: -12%). At d = 64 the softmax alone sets the pace (S of the
+// 32 nothing, 3 and 4 of 32 no better than 2. FP8 mode, one-tile form
+// (B = 2, H = 16, N = 8192 and the 16384-token GQA shape): 3 of every 16
+// is fastest (+1.2 to +1.6% against 2 of 16, which gained 1.6 and 2.9%
+// against 4 of 16, itself 0.6 to 2.4% ahead of none; 1 of 16 -2%, 6 of
+// 16 -6%, 8 of 16 -12%). At d = 64 the softmax alone sets the pace (S of the
 // next tile is computed while it runs) and its weights need twice the
 // exponential unit's time of the MMAs. With two one-tile CTAs per SM
 // (B = 4, H = 16, N = 2048): 4 of 32 gains 2 to 4% without a mask and
 // loses 2.5% causal (0 fastest there; 2 of 32 -0.6%), 8 of 32 loses 4 to 7%.
 constexpr int kPolyPer32 = 2;
-constexpr int kPolyPer16F8 = 2;
+constexpr int kPolyPer16F8 = 3;
 template <int D, int MASK>
 constexpr int poly_per32() {
   return D == 64 ? (MASK == 0 ? 4 : 0) : kPolyPer32;
