@@ -158,8 +158,8 @@ int fa_bwd_with_residual(const void* q, const void* k, const void* v, const void
  *   (about 4 bytes * B*Hq*N*(d+1)); larger shapes return FA_ERR_UNSUPPORTED
  *   before anything is launched.
  *   The first call on a device looks up the array's device address (once
- *   per device, with that device current); make that first call before any
- *   stream capture. No call allocates or frees memory.
+ *   per device, with that device current). No call allocates or frees
+ *   memory.
  *   Every call shares the array and it keeps the last call's contents; the
  *   kernels rewrite what they read before using it. Calls whose kernels
  *   overlap on the GPU (from several streams or host threads) race on the
