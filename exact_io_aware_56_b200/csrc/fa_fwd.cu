@@ -8,16 +8,23 @@
 // shared memory and are dropped, only m, l and O persist, O is written once
 // together with one logsumexp per row).
 //
-// One CTA owns two 128-row Q tiles of one (batch, query head) and streams
-// the K/V tiles of its KV head once for both. Warp roles:
-//   warps 0-3   softmax for Q tile 0, warps 4-7 for Q tile 1: one thread
-//               per query row (warp w reads tensor-memory lanes 32*(w%4)..).
-//   warp 8      TMA producer: Q tiles once, then K_j / V_j into a ring of
-//               shared-memory stages (mbarrier full / empty pairs).
-//   warp 9      tensor-memory owner and MMA issuer (one thread):
-//               S_t = Q_t K_j^T (tcgen05, both operands in shared memory),
-//               O_t += P_t V_j (tcgen05, P_t read from tensor memory).
-//   warps 10-11 idle (keep the third warpgroup whole).
+// Two forms of one kernel template (FwdCfg, parameter T = Q tiles per CTA):
+//   two-tile form (T = 2, d = 128 in bf16): one CTA per SM owns two 128-row
+//     Q tiles of one (batch, query head), streams the K/V tiles of its KV
+//     head once for both, and holds all 512 tensor-memory columns;
+//   one-tile form (T = 1, d = 64 in bf16, and the FP8 mode: 128-byte rows):
+//     one Q tile per CTA, two CTAs per SM with 256 columns each, so that one
+//     CTA's start and epilogue run under the other's key-tile loop.
+// Warp roles (w0 = 4T):
+//   warps 0 .. w0-1  softmax, one warpgroup per Q tile: one thread per query
+//                    row (warp w reads tensor-memory lanes 32*(w%4)..).
+//   warp w0          TMA producer of the Q tiles (once) and of K_j into the
+//                    K ring (mbarrier full / empty pairs).
+//   warp w0+1        tensor-memory owner and MMA issuer:
+//                    S_t = Q_t K_j^T (tcgen05, both operands in shared memory),
+//                    O_t += P_t V_j (tcgen05, P_t read from tensor memory).
+//   warp w0+2        TMA producer of V_j into the V ring.
+//   warp w0+3        idle (keeps the last warpgroup whole).
 // The softmax is the online form of the "Four ideas" list (item "Online
 // softmax"): running max m, running sum l, O rescaled by e^(m - m_new)
 // when the max grows (by more than the rescale threshold below). P_t goes
@@ -25,21 +32,25 @@
 // rescale precedes the first, and the first half's share of O_t += P_t V_j
 // runs while the second half's exponentials are computed.
 //
-// Tensor memory (512 columns x 128 lanes, fp32):
-//   [0,128) S_0 | [128,256) S_1 | [256,256+D) O_0 | [256+D,256+2D) O_1
-// P_t (bf16, two per column) overwrites the first 64 columns of S_t.
+// Tensor memory (128 lanes, fp32 columns): S_t at [128t, 128t + 128), O_t
+// at kColO + D t. P_t is written over the first columns of S_t (bf16 two
+// per column, e4m3 four per column), except at d = 64, where it has its own
+// 64 columns at kColP + 64t (the separate-P schedule below). Two-tile form:
+//   [0,128) S_0 | [128,256) S_1 | [256,384) O_0 | [384,512) O_1;
+// one-tile form: [0,128) S | [128,128+D) O | at d = 64 [192,256) P.
 //
-// Ordering argument used by the softmax warps: the MMA thread issues, for
-// each tile t, S_t^(j+1) after both halves of O_t += P_t^j V_j, and tcgen05
-// operations complete in issue order, so once S_t^(j+1) is signalled
-// complete the O_t accumulator holds every earlier product and may be
-// rescaled in place until the first half of P_t^(j+1) is handed back.
+// Ordering argument used by the softmax warps when P is written over S: the
+// MMA thread issues, for each tile t, S_t^(j+1) after both halves of
+// O_t += P_t^j V_j, and tcgen05 operations complete in issue order, so once
+// S_t^(j+1) is signalled complete the O_t accumulator holds every earlier
+// product and may be rescaled in place until the first half of P_t^(j+1) is
+// handed back.
 //
-// At d = 64 tensor memory also holds a separate P_t ([384 + 64t, +64)), and
-// the MMA thread issues S_t^(j+1) as soon as the softmax has loaded S_t^j
-// (barrier s_free), before O_t += P_t^j V_j. The softmax then waits for
-// that product's completion (barrier pv_done) before it writes P_t^(j+1) or
-// rescales O_t, instead of relying on the order above.
+// Separate-P schedule (d = 64): the MMA thread issues S_t^(j+1) as soon as
+// the softmax has loaded S_t^j (barrier s_free), before O_t += P_t^j V_j.
+// The softmax then waits for that product's completion (barrier pv_done)
+// before it writes P_t^(j+1) or rescales O_t, instead of relying on the
+// order above.
 //
 // The exponentials are base 2: scores are scaled by scale*log2(e), and
 // L = (m + log2 l) * ln 2. A warp whose rows' maxima did not grow on a tile
@@ -47,7 +58,8 @@
 //
 // Epilogue (bf16 mode): each softmax warpgroup stages its normalised O tile
 // (and the residual) in shared memory in the 128-byte-swizzled box layout
-// and writes it with TMA tensor stores (o and o_resid tensor maps).
+// and writes it with TMA tensor stores (o and o_resid tensor maps); the FP8
+// mode stores its rows from registers.
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -60,7 +72,7 @@ namespace {
 
 constexpr int kBM = 128;   // query rows per Q tile
 constexpr int kBN = 128;   // keys per K/V tile
-// One-tile form (d = 64, two CTAs per SM): register shares of the softmax
+// One-tile form (two CTAs per SM): register shares of the softmax
 // warpgroup and of the producer / MMA warpgroup (setmaxnreg), summing to
 // what a launch at 128 registers per thread gives the CTA.
 constexpr int kSoftmaxRegs1 = 192;
@@ -210,12 +222,11 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, T>::kThreads, FwdCfg<D, F8, T>::
                const __grid_constant__ CUtensorMap tmR, const FwdArgs a) {
   using C = FwdCfg<D, F8, T>;
   static_assert(!F8 || MASK != 2, "FP8 mode covers the unmasked and causal forward");
-  // Separate-P schedule: with d = 64 tensor memory has room for P next to S
-  // (S_t at [128t, 128t+128), O_t at [256 + 64t, ...), P_t at [384 + 64t,
-  // 384 + 64t + 64)), so S_t of the next key tile is computed as soon as
-  // the softmax has loaded S_t, while it still turns the scores into P, and
-  // the softmax warps never wait for P V and S to pass through the tensor
-  // pipe between tiles.
+  // Separate-P schedule: at d = 64 tensor memory has room for P next to S
+  // and O (P_t at kColP + 64t), so S_t of the next key tile is computed as
+  // soon as the softmax has loaded S_t, while it still turns the scores
+  // into P, and the softmax warps never wait for P V and S to pass through
+  // the tensor pipe between tiles.
   constexpr bool SEP = (D == 64) && !F8;
   constexpr int KS = C::kKStages;  // K ring stages
   constexpr int VS = C::kVStages;  // V ring stages
