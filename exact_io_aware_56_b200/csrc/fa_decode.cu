@@ -30,8 +30,10 @@
 // Warp roles (192 threads):
 //   warps 0-3  softmax, one thread per tensor-memory lane (Q slot).
 //   warp 4     TMA producer: K_j / V_j into a ring of stages, Q per segment.
-//   warp 5     tensor-memory owner and MMA issuer (one thread):
-//              S = Q K_j^T (both in shared memory), O += P V_j (P in TMEM).
+//   warp 5     tensor-memory owner and MMA issuer (the whole warp runs the
+//              issue loop so descriptors stay warp-uniform; one elected lane
+//              issues): S = Q K_j^T (both in shared memory), O += P V_j (P in
+//              TMEM).
 //
 // Tensor memory (512 columns allocated):
 //   [0,256) S_0, S_1 | [256,384) P_0, P_1 (bf16 pairs) | [384,...) O_0 (, O_1)
