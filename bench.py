@@ -103,9 +103,22 @@ def load_peaks():
     try:
         with open(path) as f:
             pk = json.load(f)
-        return pk, "measured"
+        if isinstance(pk, dict):
+            return pk, "measured"
     except (OSError, ValueError):
-        return dict(FALLBACK_PEAKS), "fallback"
+        pass
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def peak_value(key: str):
+    """(value, source) of one roofline denominator: the measured figure when
+    MEASURED_PEAKS.json holds a positive number under ``key``, else the
+    fallback figure, labelled as such."""
+    pk, src = load_peaks()
+    v = pk.get(key)
+    if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+        return float(v), src
+    return float(FALLBACK_PEAKS[key]), "fallback"
 
 
 def captured_traffic(kernel: str, workload: str):
@@ -601,8 +614,7 @@ def native_arm(args):
                                "flops": w.bwd_flops(), "launches_per_step": 1}
         kernels["bwd_pre"] = {"ms": statistics.mean(e[1].elapsed_time(e[2]) for e in evs)}
         kernels["bwd_post"] = {"ms": statistics.mean(e[3].elapsed_time(e[4]) for e in evs)}
-    peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_src = peak_value("bf16_tflops")
     for kn in ("fwd", "bwd_main"):
         if kn in kernels:
             kk = kernels[kn]
@@ -732,8 +744,8 @@ def fp8_native_arm(args, w):
         raise RuntimeError("device watchdog fired during the timed steps")
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     value = w.fwd_flops() * args.steps * world / (ms_total * 1e-3) / 1e12
-    peaks, peak_src = load_peaks()
-    peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_src = peak_value("bf16_tflops")
+    peak *= 2.0
     achieved = w.fwd_flops() / (ms_total / args.steps * 1e-3) / 1e12
     roofline = {
         "bound": "tensor", "kernel": "fwd_fp8", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -855,8 +867,7 @@ def decode_native_arm(args, w):
         raise RuntimeError("device watchdog fired during the timed steps")
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
     value = w.bytes_moved() * args.steps * world / (ms_total * 1e-3) / 1e9
-    peaks, peak_src = load_peaks()
-    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    peak, peak_src = peak_value("hbm_gbs")
     main_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     merge_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     # The split kernel's algorithmic bytes: it reads q and the K/V cache

@@ -136,3 +136,19 @@ def test_clock_summary_keeps_only_the_timed_window():
     assert sm["reasons"] == ["sw_power_cap"] and sm["sm_max_mhz"] == 1965.0
     c.t_begin, c.t_end = 2.1, 2.2  # shorter than the polling period: nearest sample to its middle
     assert c.summary()["samples"] == 1 and c.summary()["sm_mhz"] == 1900.0
+
+
+def test_peak_value_measured_fallback_and_malformed(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.peak_value("bf16_tflops") == (bench.FALLBACK_PEAKS["bf16_tflops"], "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6431.7, "bf16_tflops": 1656.9}))
+    assert bench.peak_value("bf16_tflops") == (1656.9, "measured")
+    assert bench.peak_value("hbm_gbs") == (6431.7, "measured")
+    # A key the file lacks, or holds as something other than a positive
+    # number, takes the fallback figure and says so.
+    assert bench.peak_value("bf16_tflops_sustained") == (bench.FALLBACK_PEAKS["bf16_tflops_sustained"],
+                                                         "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"bf16_tflops": {"burst": 1656.9}, "hbm_gbs": -1}))
+    assert bench.peak_value("bf16_tflops")[1] == "fallback" and bench.peak_value("hbm_gbs")[1] == "fallback"
+    (tmp_path / "MEASURED_PEAKS.json").write_text("[1, 2]")
+    assert bench.peak_value("hbm_gbs") == (bench.FALLBACK_PEAKS["hbm_gbs"], "fallback")
