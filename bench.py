@@ -54,10 +54,14 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    p.add_argument("--e2e-steps", type=int, default=8)
+    p.add_argument("--e2e-steps", type=int, default=None,
+                   help="end-to-end steps through the public API (default: --steps; 0 skips them)")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args(argv)
+    args = p.parse_args(argv)
+    if args.e2e_steps is None:
+        args.e2e_steps = args.steps
+    return args
 
 
 # ----------------------------------------------------------------- ranks
@@ -754,33 +758,30 @@ def fp8_native_arm(args, w):
     }
     e2e = None
     if args.e2e_steps > 0:
-        hin = {n: host[n].pin_memory() for n in ("q", "k", "v")}
-        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse)]
-        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        # bf16 q, k, v in from pinned host memory, quantized and attended on
+        # the device, o and lse back, pipelined as the training step's e2e
+        # (see pipelined_e2e). The codes and scales are one set: quantization
+        # and attention of consecutive steps run in order on one stream.
+        hin = [host[n].pin_memory() for n in ("q", "k", "v")]
+
+        def make_set():
+            return [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hin], [torch.empty_like(o),
+                                                                                    torch.empty_like(lse)]
+
+        def run(dins, douts, st):
+            fa.fa_quantize_fp8(dins[0], q8, sq, False, st)
+            fa.fa_quantize_fp8(dins[1], k8, sk, False, st)
+            fa.fa_quantize_fp8(dins[2], v8, sv, True, st)
+            fa.fa_fwd_fp8(q8, sq, k8, sk, v8, sv, douts[0], douts[1], w.causal, w.scale, st)
+
+        h2d = sum(t.numel() * t.element_size() for t in hin)
         d2h = sum(t.numel() * t.element_size() for t in (o, lse))
-
-        def e2e_step():
-            for n, t in (("q", q), ("k", k), ("v", v)):
-                t.copy_(hin[n], non_blocking=True)
-            fa.fa_quantize_fp8(q, q8, sq, False, stream)
-            fa.fa_quantize_fp8(k, k8, sk, False, stream)
-            fa.fa_quantize_fp8(v, v8, sv, True, stream)
-            step()
-            for src, dst in zip((o, lse), hout):
-                dst.copy_(src, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize(dev)
+        pipelined_e2e(dev, stream, hin, make_set, run, 2)  # warm-up of the streams and buffers
         barrier(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e_ms = max_over_ranks(pipelined_e2e(dev, stream, hin, make_set, run, args.e2e_steps), dev)
         e2e = {"value": w.fwd_flops() * args.e2e_steps * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "pipelined": "inputs of step k+1 and outputs of step k-1 cross the host link while step k computes"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         flops, secs, n, threads = fp8_oracle_sample(w, args.cpu_seconds)
