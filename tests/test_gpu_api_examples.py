@@ -14,7 +14,7 @@ from .parity import assert_close_abs, assert_close_lse
 pytestmark = pytest.mark.gpu
 
 
-def test_readme_calls():
+def test_convenience_calls_against_the_oracle():
     g = torch.Generator().manual_seed(12)
     q = torch.randn(2, 16, 384, 128, generator=g).to(torch.bfloat16).cuda()
     k = torch.randn(2, 4, 384, 128, generator=g).to(torch.bfloat16).cuda()
