@@ -113,7 +113,8 @@ constexpr float kF8Offset = 8.0f - kF8Rescale;
 // next tile is computed while it runs) and its weights need twice the
 // exponential unit's time of the MMAs. With two one-tile CTAs per SM
 // (B = 4, H = 16, N = 2048): 4 of 32 gains 2 to 4% without a mask and
-// loses 2.5% causal (0 fastest there; 2 of 32 -0.6%), 8 of 32 loses 4 to 7%.
+// loses 2.5% causal (0 fastest there; 2 of 32 -0.6%); 5 and 6 of 32 lose 1 to
+// 2.5% against 4, 8 of 32 loses 4 to 7%.
 constexpr int kPolyPer32 = 2;
 constexpr int kPolyPer16F8 = 3;
 template <int D, int MASK>
